@@ -1,0 +1,14 @@
+"""fp64 CPU oracle (test infrastructure only; see ``oracle.attention``).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline legs of
+``bench.py`` may import this package.  The CUDA library never does.
+"""
+from .attention import (  # noqa: F401
+    attn_scores_ref,
+    attn_probs_ref,
+    attn_fwd_ref,
+    attn_fwd_rows_ref,
+    attn_bwd_ref,
+    online_fwd_ref,
+    fa1_fwd_ref,
+)

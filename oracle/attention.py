@@ -1,0 +1,270 @@
+"""fp64 CPU oracle for exact scaled-dot-product attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import, call or
+execute this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it.  It shares
+no code, constant or helper with the CUDA library and imports nothing from it.
+
+What it computes (all in float64, on whatever arrays it is handed):
+
+* ``attn_fwd_ref``  -- the plain definition: S = scale * Q K^T, causal entries
+  (key j > query i) set to -inf, two-pass softmax (row max, then the sum of
+  exponentials), P = exp(S - LSE), O = P V, LSE = m + ln(sum exp(S - m)).
+  Source: marketmaker.cc "Flash Attention and the sequence-length problem",
+  section "Why attention is memory-bound" (the softmax(QK^T/sqrt(d_k))V
+  definition) and the explicit-score PyTorch snippet of section "Integration
+  is eight lines"; ultralytics.com glossary "Flash Attention", the
+  full-matrix reference line of its code listing.  The log-sum-exp is the
+  natural log of the row sum of exp(scaled scores): the pages keep a running
+  max m and running sum l per row and write back only those two numbers per
+  row (ultralytics glossary, "How Flash Attention works"); storing them as
+  m + ln l is the reading used here.
+* ``attn_bwd_ref`` -- the analytic gradient of that definition (the pages do
+  not print it; it follows from the softmax Jacobian): dV = P^T dO,
+  dP = dO V^T, D_i = sum_c dO_ic O_ic, dS = P * (dP - D), dQ = scale dS K,
+  dK = scale dS^T Q.  The recomputation of P from Q, K and the stored LSE is
+  the marketmaker.cc section "Backward pass: recompute instead of store".
+* ``online_fwd_ref`` -- the online-softmax re-association, one key/value block
+  at a time: running row max m, running sum l, unnormalised accumulator O~;
+  when the max grows, O~ and l are rescaled by exp(m_old - m_new); O = O~ / l
+  at the end.  Source: ultralytics.com glossary "Flash Attention", the
+  streaming loop of its code listing, and marketmaker.cc section "Online
+  softmax recurrence" (whose displayed equations were lost in extraction; they
+  are reconstructed from its prose, which says that whenever a block raises
+  the running maximum the output accumulated so far is multiplied by
+  e^{m^(j-1) - m^(j)}).
+* ``fa1_fwd_ref`` -- the per-step-normalised loop of the marketmaker.cc
+  section "The Flash Attention algorithm" (query blocks outer, key/value blocks
+  inner, O normalised by the running sum after every block).
+
+Row chunking: ``attn_fwd_ref`` and ``attn_bwd_ref`` may process the query rows
+in chunks (``row_chunk``) so that an N x N fp64 matrix never has to exist for
+the long configurations.  Every chunk holds complete rows, so each row is
+still computed with the plain two-pass definition; the gradient sums over rows
+(dK, dV) are just added chunk by chunk.
+
+Parity pins for every function live in ``tests/test_oracle_pins.py`` (brute
+force, closed forms, invariants, finite differences, the pages' worked
+numbers).  No function here is "parity unpinned".
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "attn_scores_ref",
+    "attn_probs_ref",
+    "attn_fwd_ref",
+    "attn_fwd_rows_ref",
+    "attn_bwd_ref",
+    "online_fwd_ref",
+    "fa1_fwd_ref",
+]
+
+
+def _f64(x):
+    return np.asarray(x, dtype=np.float64)
+
+
+def _causal_mask(rows, n_k):
+    """True where key j is in the future of query row i (j > i)."""
+    rows = np.asarray(rows)
+    return np.arange(n_k)[None, :] > rows[:, None]
+
+
+def attn_scores_ref(q, k, scale, causal=False, rows=None):
+    """S = scale * Q K^T for one head; masked entries are -inf.
+
+    q: [Nq, d], k: [Nk, d].  ``rows`` selects query rows (their absolute
+    indices are used for the causal mask).
+    """
+    q = _f64(q)
+    k = _f64(k)
+    if rows is None:
+        rows = np.arange(q.shape[0])
+    else:
+        rows = np.asarray(rows)
+        q = q[rows]
+    s = float(scale) * (q @ k.T)
+    if causal:
+        s = np.where(_causal_mask(rows, k.shape[0]), -np.inf, s)
+    return s, rows
+
+
+def _two_pass(s):
+    """Row max, then log of the row sum of exp(s - max).  Returns (lse, p)."""
+    m = s.max(axis=-1, keepdims=True)
+    # A fully masked row (never produced by square causal inputs) has m = -inf;
+    # its probabilities are 0 and its LSE is -inf.
+    m_safe = np.where(np.isfinite(m), m, 0.0)
+    e = np.exp(s - m_safe)
+    l = e.sum(axis=-1, keepdims=True)
+    with np.errstate(divide="ignore"):
+        lse = np.where(l > 0, m_safe + np.log(l), -np.inf)
+    p = np.where(l > 0, e / np.where(l > 0, l, 1.0), 0.0)
+    return lse[..., 0], p
+
+
+def attn_probs_ref(q, k, scale, causal=False):
+    """P = softmax(S) for one head (two-pass)."""
+    s, _ = attn_scores_ref(q, k, scale, causal)
+    _, p = _two_pass(s)
+    return p
+
+
+def attn_fwd_rows_ref(q, k, v, scale, causal=False, rows=None, row_chunk=1024):
+    """O and LSE for the selected query rows of one head.
+
+    q, k, v: [N, d].  Returns (o [len(rows), d], lse [len(rows)]).
+    """
+    v = _f64(v)
+    if rows is None:
+        rows = np.arange(np.asarray(q).shape[0])
+    rows = np.asarray(rows)
+    o = np.empty((rows.shape[0], v.shape[1]), dtype=np.float64)
+    lse = np.empty((rows.shape[0],), dtype=np.float64)
+    for c0 in range(0, rows.shape[0], row_chunk):
+        r = rows[c0:c0 + row_chunk]
+        s, _ = attn_scores_ref(q, k, scale, causal, rows=r)
+        lse_c, p = _two_pass(s)
+        o[c0:c0 + r.shape[0]] = p @ v
+        lse[c0:c0 + r.shape[0]] = lse_c
+    return o, lse
+
+
+def attn_fwd_ref(q, k, v, scale, causal=False, row_chunk=1024):
+    """Forward for [..., N, d] inputs (any number of leading batch/head dims).
+
+    Returns (O [..., N, d], LSE [..., N]) in float64.
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    lead = q.shape[:-2]
+    n, d = q.shape[-2:]
+    qf = q.reshape((-1, n, d))
+    kf = k.reshape((-1,) + k.shape[-2:])
+    vf = v.reshape((-1,) + v.shape[-2:])
+    o = np.empty((qf.shape[0], n, vf.shape[-1]))
+    lse = np.empty((qf.shape[0], n))
+    for h in range(qf.shape[0]):
+        o[h], lse[h] = attn_fwd_rows_ref(qf[h], kf[h], vf[h], scale, causal,
+                                         row_chunk=row_chunk)
+    return o.reshape(lead + (n, vf.shape[-1])), lse.reshape(lead + (n,))
+
+
+def attn_bwd_ref(q, k, v, do, scale, causal=False, row_chunk=1024):
+    """Analytic gradient of O = softmax(scale Q K^T [+ causal mask]) V.
+
+    Inputs [..., N, d]; returns (dQ, dK, dV) in float64.  O and P are the
+    oracle's own fp64 values (not a GPU's).
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    do = _f64(do)
+    lead = q.shape[:-2]
+    n, d = q.shape[-2:]
+    nk = k.shape[-2]
+    qf, kf, vf, dof = (x.reshape((-1,) + x.shape[-2:]) for x in (q, k, v, do))
+    dq = np.zeros_like(qf)
+    dk = np.zeros_like(kf)
+    dv = np.zeros_like(vf)
+    for h in range(qf.shape[0]):
+        for c0 in range(0, n, row_chunk):
+            rows = np.arange(c0, min(n, c0 + row_chunk))
+            s, _ = attn_scores_ref(qf[h], kf[h], scale, causal, rows=rows)
+            _, p = _two_pass(s)                     # [r, Nk]
+            o = p @ vf[h]                           # [r, d]
+            dO = dof[h, rows]                       # [r, d]
+            dv[h] += p.T @ dO                       # dV = P^T dO
+            dp = dO @ vf[h].T                       # dP = dO V^T
+            D = np.sum(dO * o, axis=-1, keepdims=True)  # D_i = sum_c dO_ic O_ic
+            ds = p * (dp - D)                       # dS = P o (dP - D)
+            dq[h, rows] = float(scale) * (ds @ kf[h])   # dQ = scale dS K
+            dk[h] += float(scale) * (ds.T @ qf[h, rows])  # dK = scale dS^T Q
+    shp = lambda x, ref: x.reshape(lead + ref.shape[-2:])
+    return shp(dq, q), shp(dk, k), shp(dv, v)
+
+
+def online_fwd_ref(q, k, v, scale, causal=False, block=128, dtype=np.float64):
+    """Online-softmax forward for one head, streaming key/value blocks.
+
+    All query rows are processed against one key/value block at a time.  After
+    block j:  m_j = max(m_{j-1}, rowmax S_j);  l_j = e^{m_{j-1}-m_j} l_{j-1} +
+    rowsum e^{S_j - m_j};  O~_j = e^{m_{j-1}-m_j} O~_{j-1} + e^{S_j - m_j} V_j.
+    Finally O = O~ / l and LSE = m + ln l.  ``dtype`` lets the same steps run
+    in float32 (the glossary's own precision) for its worked error figure.
+    """
+    q = np.asarray(q, dtype=dtype)
+    k = np.asarray(k, dtype=dtype)
+    v = np.asarray(v, dtype=dtype)
+    n, nk = q.shape[0], k.shape[0]
+    sc = dtype(scale)
+    row_max = np.full((n, 1), -np.inf, dtype=dtype)
+    row_sum = np.zeros((n, 1), dtype=dtype)
+    out = np.zeros((n, v.shape[1]), dtype=dtype)
+    rows = np.arange(n)
+    for start in range(0, nk, block):
+        stop = min(nk, start + block)
+        scores = (q @ k[start:stop].T) * sc
+        if causal:
+            cols = np.arange(start, stop)
+            scores = np.where(cols[None, :] > rows[:, None], -np.inf, scores)
+        new_max = np.maximum(row_max, scores.max(axis=-1, keepdims=True))
+        safe = np.where(np.isfinite(new_max), new_max, 0.0).astype(dtype)
+        with np.errstate(invalid="ignore"):
+            rescale = np.where(np.isfinite(new_max), np.exp(row_max - safe), 0.0).astype(dtype)
+        probs = np.exp(scores - safe)
+        row_sum = row_sum * rescale + probs.sum(axis=-1, keepdims=True)
+        out = out * rescale + probs @ v[start:stop]
+        row_max = new_max
+    with np.errstate(divide="ignore", invalid="ignore"):
+        o = np.where(row_sum > 0, out / np.where(row_sum > 0, row_sum, 1), 0.0)
+        lse = np.where(row_sum > 0, row_max + np.log(np.where(row_sum > 0, row_sum, 1)), -np.inf)
+    return o.astype(dtype), lse[:, 0].astype(dtype)
+
+
+def fa1_fwd_ref(q, k, v, scale, causal=False, block_r=128, block_c=128):
+    """The tiled loop with per-step normalisation, for one head.
+
+    For each query block: O = 0, m = -inf, l = 0.  For each key/value block:
+    S = scale Q_i K_j^T, m_ij = rowmax S, P = exp(S - m_ij), l_ij = rowsum P,
+    m_new = max(m, m_ij), l_new = e^{m - m_new} l + e^{m_ij - m_new} l_ij,
+    O = O (l e^{m - m_new} / l_new) + (P V_j) (e^{m_ij - m_new} / l_new),
+    then m = m_new, l = l_new.  Returns (O, LSE = m + ln l).
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    n, nk = q.shape[0], k.shape[0]
+    o_all = np.zeros((n, v.shape[1]))
+    lse_all = np.zeros((n,))
+    for r0 in range(0, n, block_r):
+        rows = np.arange(r0, min(n, r0 + block_r))
+        o = np.zeros((rows.shape[0], v.shape[1]))
+        m = np.full((rows.shape[0], 1), -np.inf)
+        l = np.zeros((rows.shape[0], 1))
+        for c0 in range(0, nk, block_c):
+            cols = np.arange(c0, min(nk, c0 + block_c))
+            s = float(scale) * (q[rows] @ k[cols].T)
+            if causal:
+                s = np.where(cols[None, :] > rows[:, None], -np.inf, s)
+            m_ij = s.max(axis=-1, keepdims=True)
+            fin_ij = np.isfinite(m_ij)
+            p = np.where(fin_ij, np.exp(s - np.where(fin_ij, m_ij, 0.0)), 0.0)
+            l_ij = p.sum(axis=-1, keepdims=True)
+            m_new = np.maximum(m, m_ij)
+            fin_new = np.isfinite(m_new)
+            mn = np.where(fin_new, m_new, 0.0)
+            a_old = np.where(np.isfinite(m), np.exp(m - mn), 0.0)
+            a_blk = np.where(fin_ij, np.exp(np.where(fin_ij, m_ij, 0.0) - mn), 0.0)
+            l_new = a_old * l + a_blk * l_ij
+            safe_l = np.where(l_new > 0, l_new, 1.0)
+            o = o * (l * a_old / safe_l) + (p @ v[cols]) * (a_blk / safe_l)
+            m, l = m_new, l_new
+        o_all[rows] = o
+        lse_all[rows] = (m + np.log(np.where(l > 0, l, 1.0)))[:, 0]
+    return o_all, lse_all
+

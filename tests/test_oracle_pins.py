@@ -1,0 +1,342 @@
+"""Pins for the fp64 oracle, each against something other than the oracle.
+
+* brute force: pure-Python loops over math.exp on tiny inputs;
+* a library routine: scipy.special.softmax / logsumexp for the special case
+  of one query row;
+* closed forms and invariants of softmax attention;
+* finite differences of an independent (pure-Python) forward for the
+  gradient;
+* the pages' own worked numbers (tests/golden/).
+
+Each is chosen so that a plausible slip in the oracle (a dropped term, a wrong
+sign or index, a transposed operand, a wrong mask direction) fails at least
+one of them.
+"""
+
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+from oracle import (attn_bwd_ref, attn_fwd_ref, attn_fwd_rows_ref,
+                    attn_probs_ref, attn_scores_ref, fa1_fwd_ref,
+                    online_fwd_ref)
+from exact_io_aware_84_b200.metrics import score_matrix_bytes
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _brute_fwd(q, k, v, scale, causal):
+    """Explicit loops: for every query row, every key, every channel."""
+    n, d = len(q), len(q[0])
+    nk, dv = len(k), len(v[0])
+    o = [[0.0] * dv for _ in range(n)]
+    lse = [0.0] * n
+    for i in range(n):
+        s = []
+        for j in range(nk):
+            if causal and j > i:
+                continue
+            dot = 0.0
+            for c in range(d):
+                dot += float(q[i][c]) * float(k[j][c])
+            s.append((j, scale * dot))
+        mx = max(x for _, x in s)
+        tot = sum(math.exp(x - mx) for _, x in s)
+        lse[i] = mx + math.log(tot)
+        for j, x in s:
+            w = math.exp(x - mx) / tot
+            for c in range(dv):
+                o[i][c] += w * float(v[j][c])
+    return np.array(o), np.array(lse)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n,d", [(1, 1), (2, 3), (5, 4), (8, 2), (8, 4)])
+def test_forward_matches_brute_force(n, d, causal):
+    r = _rng(100 * n + d + causal)
+    q, k, v = (r.standard_normal((n, d)) for _ in range(3))
+    scale = 0.7
+    o_b, lse_b = _brute_fwd(q, k, v, scale, causal)
+    o, lse = attn_fwd_ref(q, k, v, scale, causal)
+    np.testing.assert_allclose(o, o_b, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lse, lse_b, rtol=0, atol=1e-14)
+
+
+def test_forward_matches_brute_force_rectangular_keys():
+    # more keys than queries, non-causal: a transposed q/k operand would fail
+    r = _rng(7)
+    q = r.standard_normal((3, 4))
+    k = r.standard_normal((6, 4))
+    v = r.standard_normal((6, 2))
+    o_b, lse_b = _brute_fwd(q, k, v, 0.3, False)
+    o, lse = attn_fwd_rows_ref(q, k, v, 0.3, False)
+    np.testing.assert_allclose(o, o_b, atol=1e-14)
+    np.testing.assert_allclose(lse, lse_b, atol=1e-14)
+
+
+def test_batched_leading_dims_match_per_head():
+    r = _rng(11)
+    q, k, v = (r.standard_normal((2, 3, 9, 5)) for _ in range(3))
+    o, lse = attn_fwd_ref(q, k, v, 0.5, True)
+    for b in range(2):
+        for h in range(3):
+            ob, lb = _brute_fwd(q[b, h], k[b, h], v[b, h], 0.5, True)
+            np.testing.assert_allclose(o[b, h], ob, atol=1e-14)
+            np.testing.assert_allclose(lse[b, h], lb, atol=1e-14)
+
+
+def test_single_row_is_library_softmax():
+    # one query row: P is scipy's softmax of the scaled scores, LSE its logsumexp
+    r = _rng(3)
+    q = r.standard_normal((1, 16))
+    k = r.standard_normal((40, 16))
+    v = r.standard_normal((40, 8))
+    scale = 1 / 4
+    s = scale * (k @ q[0])
+    p_lib = scipy.special.softmax(s)
+    o, lse = attn_fwd_ref(q, k, v, scale, False)
+    np.testing.assert_allclose(lse[0], scipy.special.logsumexp(s), atol=1e-13)
+    np.testing.assert_allclose(o[0], p_lib @ v, atol=1e-13)
+    np.testing.assert_allclose(attn_probs_ref(q, k, scale)[0], p_lib, atol=1e-15)
+
+
+def test_row_chunking_does_not_change_results():
+    r = _rng(5)
+    q, k, v, do = (r.standard_normal((2, 37, 6)) for _ in range(4))
+    o1, l1 = attn_fwd_ref(q, k, v, 0.4, True, row_chunk=1000)
+    o2, l2 = attn_fwd_ref(q, k, v, 0.4, True, row_chunk=5)
+    np.testing.assert_allclose(o1, o2, atol=1e-15)
+    np.testing.assert_allclose(l1, l2, atol=1e-15)
+    g1 = attn_bwd_ref(q, k, v, do, 0.4, True, row_chunk=1000)
+    g2 = attn_bwd_ref(q, k, v, do, 0.4, True, row_chunk=4)
+    for a, b in zip(g1, g2):
+        np.testing.assert_allclose(a, b, atol=1e-13)
+
+
+def test_sampled_rows_match_full():
+    r = _rng(6)
+    q, k, v = (r.standard_normal((50, 8)) for _ in range(3))
+    rows = np.array([0, 1, 17, 31, 49])
+    o, lse = attn_fwd_ref(q, k, v, 0.3, True)
+    os_, ls = attn_fwd_rows_ref(q, k, v, 0.3, True, rows=rows, row_chunk=2)
+    np.testing.assert_allclose(os_, o[rows], atol=1e-15)
+    np.testing.assert_allclose(ls, lse[rows], atol=1e-15)
+
+
+# ---------------------------------------------------------------- invariants
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_probability_rows_sum_to_one(causal):
+    r = _rng(8)
+    q, k = r.standard_normal((33, 7)), r.standard_normal((33, 7))
+    p = attn_probs_ref(q, k, 0.9, causal)
+    np.testing.assert_allclose(p.sum(-1), 1.0, atol=1e-14)
+    assert (p >= 0).all()
+    if causal:
+        assert np.all(np.triu(p, 1) == 0)
+        assert np.all(np.diag(p) > 0)
+
+
+def test_zero_query_gives_column_means():
+    r = _rng(9)
+    n = 21
+    q = np.zeros((n, 5))
+    k, v = r.standard_normal((n, 5)), r.standard_normal((n, 3))
+    o, lse = attn_fwd_ref(q, k, v, 0.5, False)
+    np.testing.assert_allclose(o, np.broadcast_to(v.mean(0), o.shape), atol=1e-14)
+    np.testing.assert_allclose(lse, math.log(n), atol=1e-14)
+    o, lse = attn_fwd_ref(q, k, v, 0.5, True)
+    cum = np.cumsum(v, 0) / np.arange(1, n + 1)[:, None]
+    np.testing.assert_allclose(o, cum, atol=1e-14)
+    np.testing.assert_allclose(lse, np.log(np.arange(1, n + 1)), atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_constant_value_rows(causal):
+    r = _rng(10)
+    q, k = r.standard_normal((19, 4)), r.standard_normal((19, 4))
+    c = r.standard_normal(6)
+    v = np.broadcast_to(c, (19, 6)).copy()
+    o, _ = attn_fwd_ref(q, k, v, 1.3, causal)
+    np.testing.assert_allclose(o, np.broadcast_to(c, o.shape), atol=1e-14)
+
+
+def test_causal_first_row():
+    r = _rng(12)
+    q, k, v = (r.standard_normal((10, 4)) for _ in range(3))
+    o, lse = attn_fwd_ref(q, k, v, 0.6, True)
+    np.testing.assert_allclose(o[0], v[0], atol=1e-15)
+    np.testing.assert_allclose(lse[0], 0.6 * q[0] @ k[0], atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_shift_invariance(causal):
+    # adding the same vector u to every key adds scale*q_i.u to row i's scores
+    r = _rng(13)
+    q, k, v = (r.standard_normal((15, 4)) for _ in range(3))
+    u = r.standard_normal(4)
+    o1, l1 = attn_fwd_ref(q, k, v, 0.8, causal)
+    o2, l2 = attn_fwd_ref(q, k + u, v, 0.8, causal)
+    np.testing.assert_allclose(o2, o1, atol=1e-13)
+    np.testing.assert_allclose(l2, l1 + 0.8 * (q @ u), atol=1e-13)
+
+
+def test_joint_key_value_permutation_invariance():
+    r = _rng(14)
+    q, k, v = (r.standard_normal((12, 4)) for _ in range(3))
+    perm = r.permutation(12)
+    o1, l1 = attn_fwd_ref(q, k, v, 0.8, False)
+    o2, l2 = attn_fwd_ref(q, k[perm], v[perm], 0.8, False)
+    np.testing.assert_allclose(o2, o1, atol=1e-14)
+    np.testing.assert_allclose(l2, l1, atol=1e-14)
+
+
+def test_two_keys_is_logistic():
+    # one query, two keys: weight on key 0 is sigmoid(s0 - s1)
+    q = np.array([[0.3, -1.2]])
+    k = np.array([[1.0, 0.5], [-0.4, 2.0]])
+    v = np.array([[2.0], [-3.0]])
+    s0, s1 = 0.5 * q[0] @ k[0], 0.5 * q[0] @ k[1]
+    w0 = 1 / (1 + math.exp(-(s0 - s1)))
+    o, lse = attn_fwd_ref(q, k, v, 0.5, False)
+    np.testing.assert_allclose(o[0, 0], w0 * 2.0 + (1 - w0) * -3.0, atol=1e-15)
+    np.testing.assert_allclose(lse[0], math.log(math.exp(s0) + math.exp(s1)), atol=1e-15)
+
+
+# ------------------------------------------------------ online / tiled forms
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("block", [1, 3, 64, 128, 300])
+def test_online_matches_two_pass(block, causal):
+    r = _rng(15)
+    q, k, v = (r.standard_normal((300, 16)) for _ in range(3))
+    o, lse = attn_fwd_ref(q, k, v, 0.25, causal)
+    o2, lse2 = online_fwd_ref(q, k, v, 0.25, causal, block=block)
+    np.testing.assert_allclose(o2, o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse2, lse, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("br,bc", [(1, 1), (3, 5), (128, 128), (64, 256)])
+def test_per_step_normalised_loop_matches_two_pass(br, bc, causal):
+    r = _rng(16)
+    q, k, v = (r.standard_normal((203, 8)) for _ in range(3))
+    o, lse = attn_fwd_ref(q, k, v, 0.35, causal)
+    o2, lse2 = fa1_fwd_ref(q, k, v, 0.35, causal, block_r=br, block_c=bc)
+    np.testing.assert_allclose(o2, o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse2, lse, rtol=0, atol=1e-12)
+
+
+def test_online_handles_large_scores():
+    # scores of order 1e3 would overflow a naive exp; the recurrence must not
+    r = _rng(17)
+    q, k, v = (r.standard_normal((40, 8)) * 12 for _ in range(3))
+    o, lse = attn_fwd_ref(q, k, v, 1.0, True)
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    o2, lse2 = online_fwd_ref(q, k, v, 1.0, True, block=7)
+    np.testing.assert_allclose(o2, o, atol=1e-11)
+    np.testing.assert_allclose(lse2, lse, rtol=1e-14, atol=1e-11)
+
+
+def test_glossary_fp32_loop_error_magnitude():
+    """The glossary's float32 online loop differs from float32 full-matrix
+    attention by rounding only (tests/golden/online_loop_fp32_error.txt)."""
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "online_loop_fp32_error.txt"))
+            if l.strip() and not l.startswith("#")]
+    n, d, block, seed, page, factor = rows[0]
+    n, d, block, seed, page, factor = int(n), int(d), int(block), int(seed), float(page), float(factor)
+    torch.manual_seed(seed)
+    q, k, v = torch.randn(3, n, d).unbind(0)
+    full = (torch.softmax(q @ k.T / d ** 0.5, dim=-1) @ v).numpy()
+    o32, _ = online_fwd_ref(q.numpy(), k.numpy(), v.numpy(), 1.0 / d ** 0.5,
+                            block=block, dtype=np.float32)
+    err = float(np.abs(o32.astype(np.float64) - full).max())
+    assert page / factor <= err <= page * factor, err
+
+
+# ----------------------------------------------------------------- gradient
+
+def _fd_grads(q, k, v, do, scale, causal, h=1e-6):
+    """Central differences of L = sum(dO * O) using the brute-force forward."""
+    grads = []
+    for x in (q, k, v):
+        g = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + h
+            op, _ = _brute_fwd(q, k, v, scale, causal)
+            x[idx] = old - h
+            om, _ = _brute_fwd(q, k, v, scale, causal)
+            x[idx] = old
+            g[idx] = np.sum(do * (op - om)) / (2 * h)
+        grads.append(g)
+    return grads
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n,d", [(4, 3), (7, 2), (16, 4)])
+def test_gradient_matches_finite_differences(n, d, causal):
+    r = _rng(200 + n + causal)
+    q, k, v, do = (r.standard_normal((n, d)) for _ in range(4))
+    scale = 0.6
+    dq, dk, dv = attn_bwd_ref(q, k, v, do, scale, causal)
+    for name, ana, num in zip("qkv", (dq, dk, dv), _fd_grads(q, k, v, do, scale, causal)):
+        rel = np.linalg.norm(ana - num) / max(np.linalg.norm(num), 1e-30)
+        assert rel <= 1e-6, (name, rel)
+        np.testing.assert_allclose(ana, num, rtol=1e-5, atol=1e-7)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gradient_invariants(causal):
+    r = _rng(18)
+    q, k, v, do = (r.standard_normal((2, 3, 29, 8)) for _ in range(4))
+    dq, dk, dv = attn_bwd_ref(q, k, v, do, 0.4, causal)
+    # rows of dS sum to zero, so the key gradients sum to zero over keys
+    np.testing.assert_allclose(dk.sum(-2), 0.0, atol=1e-12)
+    # every row of P sums to one, so dV summed over keys is dO summed over rows
+    np.testing.assert_allclose(dv.sum(-2), do.sum(-2), atol=1e-12)
+
+
+def test_constant_value_has_no_score_gradient():
+    r = _rng(19)
+    q, k = r.standard_normal((17, 4)), r.standard_normal((17, 4))
+    do = r.standard_normal((17, 5))
+    v = np.broadcast_to(r.standard_normal(5), (17, 5)).copy()
+    dq, dk, _ = attn_bwd_ref(q, k, v, do, 0.9, True)
+    np.testing.assert_allclose(dq, 0.0, atol=1e-13)
+    np.testing.assert_allclose(dk, 0.0, atol=1e-13)
+
+
+def test_causal_mask_direction():
+    # with causal masking, row i never depends on keys/values after i
+    r = _rng(20)
+    q, k, v = (r.standard_normal((9, 3)) for _ in range(3))
+    o1, l1 = attn_fwd_ref(q, k, v, 1.0, True)
+    k2, v2 = k.copy(), v.copy()
+    k2[5:] += 3.0
+    v2[5:] -= 2.0
+    o2, l2 = attn_fwd_ref(q, k2, v2, 1.0, True)
+    np.testing.assert_allclose(o2[:5], o1[:5], atol=0)
+    np.testing.assert_allclose(l2[:5], l1[:5], atol=0)
+    assert np.abs(o2[5:] - o1[5:]).max() > 1e-3
+    s, _ = attn_scores_ref(q, k, 1.0, True)
+    assert np.isneginf(s[0, 1]) and np.isfinite(s[1, 0])
+
+
+# ---------------------------------------------------------- pages' figures
+
+def test_score_matrix_memory_worked_examples():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "score_matrix_memory.txt"))
+            if l.strip() and not l.startswith("#")]
+    for B, H, s, e, expect, page_gb, tol in rows:
+        got = score_matrix_bytes(int(B), int(H), int(s), int(e))
+        assert got == int(expect)
+        assert abs(got / 1e9 - float(page_gb)) <= float(tol) * float(page_gb)
