@@ -1,0 +1,396 @@
+#!/usr/bin/env python
+"""Benchmark: attention forward + backward TFLOP/s on B200 through libfa.so.
+
+One step = the whole hot path over one batch: fa_fwd (O, LSE) then fa_bwd
+(dQ, dK, dV) on seeded synthetic inputs of the named workload.  FLOPs per
+step follow the pages' convention: 4 B H N^2 d for the forward (halved when
+causal) and 2.5x that for the backward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the fp64 CPU oracle, timed as is
+
+Prints one JSON line (rank 0).  Timing: W untimed warm-up steps, then K
+steps bracketed by a barrier and a device synchronize; each step's kernels
+are timed with CUDA events on the launching stream; L2 is flushed (a 256 MiB
+write) between steps, outside the events.  For N > 1 every rank runs the
+same per-GPU workload (weak scaling: attention heads are independent, so no
+data-path collective exists) and the time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "gpt2_batch"  # B=8 H=12 N=1024 d=64 bf16 causal, forward + backward
+METRIC = "attention fwd/bwd TFLOP/s on 1 B200 (bf16); % of dense BF16 tensor peak"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"bf16_tflops": float(d["bf16_tflops"]), "bf16_tflops_sustained": float(d["bf16_tflops_sustained"]),
+                "hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+# ------------------------------------------------------------------ dist
+
+def _dist_init(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ oracle leg
+
+def _oracle_sample(w, budget_s, seed=0):
+    """Time the fp64 oracle (forward + backward) on whole heads of the
+    workload until ~budget_s of CPU work; returns (TFLOP/s, heads, seconds)."""
+    import numpy as np
+    from exact_io_aware_84_b200.inputs import make_inputs
+    from exact_io_aware_84_b200.metrics import attn_bwd_flops, attn_fwd_flops
+    from oracle import attn_bwd_ref, attn_fwd_ref
+    one = w.with_(B=1, H=1, seed=seed)
+    x = make_inputs(one, with_grad=w.backward)
+    q, k, v = (x[n][0, 0].double().numpy() for n in ("q", "k", "v"))
+    do = x["do"][0, 0].double().numpy() if w.backward else None
+    flops_head = attn_fwd_flops(1, 1, w.N, w.d, w.causal) + (attn_bwd_flops(1, 1, w.N, w.d, w.causal) if w.backward else 0)
+    heads, t0 = 0, time.perf_counter()
+    while True:
+        attn_fwd_ref(q, k, v, w.scale, w.causal)
+        if w.backward:
+            attn_bwd_ref(q, k, v, do, w.scale, w.causal)
+        heads += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or heads >= w.B * w.H:
+            break
+    return flops_head * heads / el / 1e12, heads, el
+
+
+def _cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def run_reference(args):
+    """--impl reference: the fp64 CPU oracle, as it stands, on the host cores."""
+    rank, world, _ = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), 0
+    if rank != 0:
+        return 0
+    from exact_io_aware_84_b200.inputs import workload
+    w = workload(args.workload)
+    per_step_budget = max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        _oracle_sample(w, per_step_budget / 4)
+    vals, secs, heads = [], 0.0, 0
+    for _ in range(args.steps):
+        v, h, el = _oracle_sample(w, per_step_budget)
+        vals.append(v)
+        secs += el
+        heads += h
+    value = statistics.median(vals)
+    cores = _cpu_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config(w, world),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{heads} whole (b,h) heads of {w.name} (fp64 forward"
+                                   f"{' + backward' if w.backward else ''}) over {args.steps} steps"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(w, world):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+            "dtype": w.dtype, "backward": w.backward, "per_gpu": True, "parallelism": f"replicas x{world}",
+            "l2": "flushed between steps (256 MiB write)"}
+
+
+# ------------------------------------------------------------------ native leg
+
+def run_native(args):
+    import torch
+
+    import exact_io_aware_84_b200 as fa
+    from exact_io_aware_84_b200.inputs import make_inputs, workload
+    from exact_io_aware_84_b200.metrics import attn_bwd_flops, attn_fwd_flops
+
+    rank, world, local = _dist_init(args)
+    w = workload(args.workload)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    fa.load_library()
+    x = make_inputs(w.with_(seed=w.seed + rank), with_grad=w.backward)
+    g = {k: v.to(dev) for k, v in x.items()}
+    B, H, N, d = w.B, w.H, w.N, w.d
+    o = torch.empty_like(g["q"])
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    if w.backward:
+        dq, dk, dv = (torch.empty_like(g["q"]) for _ in range(3))
+        ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.fa_fwd(g["q"], g["k"], g["v"], o, lse, scale=w.scale, causal=w.causal, stream=stream)
+        ev_mid.record(stream)
+        if w.backward:
+            fa.fa_bwd(g["q"], g["k"], g["v"], o, g["do"], lse, dq, dk, dv, ws, scale=w.scale,
+                      causal=w.causal, stream=stream)
+
+    launches_per_step = 1 + (3 if w.backward else 0)
+    f_fwd = attn_fwd_flops(B, H, N, d, w.causal)
+    f_bwd = attn_bwd_flops(B, H, N, d, w.causal) if w.backward else 0.0
+    flops = f_fwd + f_bwd
+
+    ev_mid = torch.cuda.Event(enable_timing=True)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if fa.fa_last_device_status(stream) != fa.FA_OK:
+        raise RuntimeError("device status not OK after warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    _barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            ev_mid = mids[i]
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    _barrier(world)
+    status = fa.fa_last_device_status(stream)
+    if status != fa.FA_OK:
+        raise RuntimeError(f"device status {fa.fa_status_string(status)}")
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    fwd_ms = [s.elapsed_time(m) for s, m in zip(starts, mids)]
+    bwd_ms = [m.elapsed_time(e) for m, e in zip(mids, ends)]
+    total_ms = _max_over_ranks(sum(step_ms), world)
+    ms_per_step = total_ms / args.steps
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    clocks = clk.summary()
+
+    # dominant kernel (the backward launch group when present, else the forward)
+    peaks = _peaks()
+    if w.backward:
+        dom_ms, dom_flops, dom_name = statistics.mean(bwd_ms), f_bwd, "fa_bwd (prep + main + dQ convert launches)"
+    else:
+        dom_ms, dom_flops, dom_name = statistics.mean(fwd_ms), f_fwd, "fa_fwd_kernel"
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": _ncu_traffic(w.name, dom_name),
+                "peak_source": f"{peaks['source']} bf16 burst", "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                "fwd_tflops": f_fwd / (statistics.mean(fwd_ms) * 1e-3) / 1e12,
+                "bwd_tflops": (f_bwd / (statistics.mean(bwd_ms) * 1e-3) / 1e12) if w.backward else None}
+
+    # end to end through the public API: pinned host inputs -> device -> step -> host
+    e2e = None
+    if not args.no_e2e:
+        e2e = _e2e(fa, torch, w, x, dev, stream, flops, world, args)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
+        "config": _config(w, world), "roofline": roofline, "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+        "fwd_ms": statistics.mean(fwd_ms), "bwd_ms": statistics.mean(bwd_ms) if w.backward else None,
+        "pct_of_peak": {"measured_burst": value / world / peaks["bf16_tflops"],
+                        "measured_sustained": value / world / peaks["bf16_tflops_sustained"],
+                        "datasheet_2250": value / world / 2250.0},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, heads, el = _oracle_sample(w, 12.0)
+        line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": _cpu_threads(), "kind": "oracle",
+                                "sample": f"{heads} whole (b,h) heads of {w.name}, fp64 forward"
+                                          f"{' + backward' if w.backward else ''}, {el:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def _e2e(fa, torch, w, x, dev, stream, flops, world, args):
+    pin = {k: v.pin_memory() for k, v in x.items()}
+    B, H, N, d = w.B, w.H, w.N, w.d
+    outs_host = {"o": torch.empty_like(pin["q"]).pin_memory(),
+                 "lse": torch.empty((B, H, N), dtype=torch.float32).pin_memory()}
+    if w.backward:
+        for n in ("dq", "dk", "dv"):
+            outs_host[n] = torch.empty_like(pin["q"]).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs_host.values())
+
+    def one():
+        g = {k: v.to(dev, non_blocking=True) for k, v in pin.items()}
+        o, lse = fa.fa_fwd(g["q"], g["k"], g["v"], scale=w.scale, causal=w.causal, stream=stream)
+        outs_host["o"].copy_(o, non_blocking=True)
+        outs_host["lse"].copy_(lse, non_blocking=True)
+        if w.backward:
+            dq, dk, dv = fa.fa_bwd(g["q"], g["k"], g["v"], o, g["do"], lse, scale=w.scale, causal=w.causal,
+                                   stream=stream)
+            outs_host["dq"].copy_(dq, non_blocking=True)
+            outs_host["dk"].copy_(dk, non_blocking=True)
+            outs_host["dv"].copy_(dv, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        one()
+    torch.cuda.synchronize()
+    _barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(args.steps):
+        one()
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = _max_over_ranks(s.elapsed_time(e), world) / args.steps
+    return {"value": flops * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def _ncu_traffic(workload_name, kernel_name):
+    """DRAM bytes per launch from a committed ncu summary, when one exists for
+    this workload and the current kernels (else null)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d.get(workload_name, {}).get("dram_bytes_per_launch")
+    except Exception:
+        return None
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

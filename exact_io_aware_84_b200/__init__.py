@@ -1,0 +1,217 @@
+"""Exact IO-aware attention for B200 (sm_100a): Python binding of libfa.so.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libfa.so`` (see ``include/fa.h``).  PyTorch provides device
+memory and streams.  There is no fallback: if the library is missing or no
+sm_100 device is present, the calls raise.
+
+    o, lse = fa_fwd(q, k, v, causal=True)              # q,k,v: [B,H,N,d] cuda bf16/fp16
+    dq, dk, dv = fa_bwd(q, k, v, o, do, lse, causal=True)
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+__all__ = [
+    "FAError",
+    "library_path",
+    "load_library",
+    "fa_fwd",
+    "fa_bwd",
+    "fa_bwd_workspace_size",
+    "fa_status_string",
+    "fa_last_device_status",
+    "fa_debug_set_wait_limit_ms",
+    "fa_debug_set_flags",
+    "fa_version",
+    "FA_OK",
+    "FA_ERR_INVALID_ARG",
+    "FA_ERR_UNSUPPORTED",
+    "FA_ERR_MISALIGNED",
+    "FA_ERR_CUDA",
+    "FA_ERR_TIMEOUT",
+    "FA_ERR_WORKSPACE",
+    "FA_ERR_NO_DEVICE",
+    "EXPORTED_SYMBOLS",
+]
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_MISALIGNED = 3
+FA_ERR_CUDA = 4
+FA_ERR_TIMEOUT = 5
+FA_ERR_WORKSPACE = 6
+FA_ERR_NO_DEVICE = 7
+
+FA_BF16 = 0
+FA_FP16 = 1
+
+_c_int, _c_float, _vp, _sz = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+
+# name -> (restype, argtypes); mirrors include/fa.h
+_SIGNATURES = {
+    "fa_fwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _vp]),
+    "fa_bwd_workspace_size": (_sz, [_c_int, _c_int, _c_int, _c_int]),
+    "fa_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                        _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _vp]),
+    "fa_status_string": (ctypes.c_char_p, [_c_int]),
+    "fa_last_device_status": (_c_int, [_vp]),
+    "fa_debug_set_wait_limit_ms": (_c_int, [_c_int]),
+    "fa_debug_set_flags": (_c_int, [_c_int]),
+    "fa_version": (ctypes.c_char_p, []),
+}
+EXPORTED_SYMBOLS = tuple(_SIGNATURES)
+
+_LIB = None
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_status_name(status)} ({status})")
+
+
+def library_path() -> str:
+    return os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
+
+
+def load_library():
+    """Load libfa.so (built in-tree by ``python -m exact_io_aware_84_b200.build``)."""
+    global _LIB
+    if _LIB is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise FileNotFoundError(
+                f"{path} is missing: build it with `python -m exact_io_aware_84_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+def _status_name(status: int) -> str:
+    try:
+        return load_library().fa_status_string(int(status)).decode()
+    except Exception:  # the library itself may be what is missing
+        return f"status {status}"
+
+
+def fa_status_string(status: int) -> str:
+    return load_library().fa_status_string(int(status)).decode()
+
+
+def fa_version() -> str:
+    return load_library().fa_version().decode()
+
+
+def fa_debug_set_wait_limit_ms(ms: int) -> int:
+    return load_library().fa_debug_set_wait_limit_ms(int(ms))
+
+
+def fa_debug_set_flags(flags: int) -> int:
+    return load_library().fa_debug_set_flags(int(flags))
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle(stream) -> Optional[int]:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def fa_last_device_status(stream=None) -> int:
+    return load_library().fa_last_device_status(_stream_handle(stream))
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    if t.dtype == torch.float16:
+        return FA_FP16
+    raise TypeError(f"unsupported dtype {t.dtype}: expected bfloat16 or float16")
+
+
+def _check_bhnd(name, t, ref=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != 4:
+        raise ValueError(f"{name} must be [B, H, N, d], got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ref is not None and (t.shape != ref.shape or t.dtype != ref.dtype or t.device != ref.device):
+        raise ValueError(f"{name} must match q in shape, dtype and device")
+
+
+def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: bool = False, stream=None):
+    """O = softmax(scale Q K^T [causal]) V and LSE (float32, natural log).
+
+    q, k, v: [B, H, N, d] contiguous CUDA tensors (bf16 or fp16).  ``o`` and
+    ``lse`` may be preallocated ([B,H,N,d] same dtype; [B,H,N] float32).
+    """
+    torch = _torch()
+    _check_bhnd("q", q)
+    _check_bhnd("k", k, q)
+    _check_bhnd("v", v, q)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    if o is None:
+        o = torch.empty_like(q)
+    else:
+        _check_bhnd("o", o, q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    elif lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B, H, N] tensor")
+    st = load_library().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                               B, H, N, d, float(scale), int(bool(causal)), _dtype_code(q),
+                               _stream_handle(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd")
+    return o, lse
+
+
+def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(load_library().fa_bwd_workspace_size(int(B), int(H), int(N), int(d)))
+
+
+def fa_bwd(q, k, v, o, do, lse, dq=None, dk=None, dv=None, workspace=None,
+           scale: Optional[float] = None, causal: bool = False, stream=None):
+    """dQ, dK, dV of L with dL/dO = ``do``, recomputing P from Q, K and LSE."""
+    torch = _torch()
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _check_bhnd(name, t, None if name == "q" else q)
+    B, H, N, d = q.shape
+    if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B, H, N] tensor")
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_bhnd(name, t, q)
+    need = fa_bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = load_library().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                               lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                               workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                               B, H, N, d, float(scale), int(bool(causal)), _dtype_code(q),
+                               _stream_handle(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd")
+    return dq, dk, dv

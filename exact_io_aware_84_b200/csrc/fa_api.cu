@@ -1,0 +1,233 @@
+// C-ABI front end of libfa.so: argument checks, TMA descriptor encoding and
+// kernel dispatch.  See include/fa.h for the contract of every entry point.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+// Device status word: 0 = OK, else the fa_status of a kernel that gave up.
+__device__ int g_device_status = 0;
+
+namespace {
+
+int* status_ptr() {
+  int* ptr = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_device_status) != cudaSuccess) return nullptr;
+  return ptr;
+}
+
+std::atomic<int> g_wait_limit_ms{1000};
+std::atomic<int> g_debug_flags{0};
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [bh, n, d] 16-bit tensor, tile box = 64 columns x `rows` rows, 128-byte
+// swizzle; rows past n (and columns past d) read as zero.
+int encode_tile_map(CUtensorMap* m, const void* ptr, int bh, int n, int d, bool bf16, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return FA_ERR_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)bh};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)n * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                  const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  bool sm100 = false;
+};
+
+int device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_NO_DEVICE;
+  static DeviceInfo cache[64];
+  static std::once_flag flags[64];
+  if (dev < 0 || dev >= 64) return FA_ERR_NO_DEVICE;
+  std::call_once(flags[dev], [dev] {
+    int major = 0, minor = 0, sms = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev].sms = sms;
+    cache[dev].sm100 = (major == 10 && minor == 0);
+  });
+  *out = cache[dev];
+  return out->sm100 ? FA_OK : FA_ERR_NO_DEVICE;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int B, int H, int N, int d, float scale, int dtype) {
+  if (B <= 0 || H <= 0 || N <= 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || scale > 3.0e38f) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_UNSUPPORTED;
+  const long long total = (long long)B * H * ((long long)N + 255) * d;
+  if (total >= (1ll << 31)) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+uint64_t wait_limit_ns() { return (uint64_t)g_wait_limit_ms.load() * 1000000ull; }
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_version(void) { return "fa-sm100 0.1"; }
+
+const char* fa_status_string(int s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_NO_DEVICE: return "FA_ERR_NO_DEVICE";
+    default: return "FA_ERR_UNKNOWN";
+  }
+}
+
+int fa_debug_set_wait_limit_ms(int ms) {
+  if (ms < 1) return FA_ERR_INVALID_ARG;
+  g_wait_limit_ms.store(ms);
+  return FA_OK;
+}
+
+int fa_debug_set_flags(int flags) {
+  if (flags < 0) return FA_ERR_INVALID_ARG;
+  g_debug_flags.store(flags);
+  return FA_OK;
+}
+
+int fa_last_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  return v;
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+           float scale, int causal, int dtype, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  int st = check_common(B, H, N, d, scale, dtype);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_MISALIGNED;
+  DeviceInfo di;
+  if ((st = device_info(&di)) != FA_OK) return st;
+  const bool bf16 = dtype == FA_BF16;
+  const int bh = B * H;
+  CUtensorMap tq, tk, tv;
+  if (encode_tile_map(&tq, q, bh, N, d, bf16, kBlockM) != FA_OK ||
+      encode_tile_map(&tk, k, bh, N, d, bf16, kBlockN) != FA_OK ||
+      encode_tile_map(&tv, v, bh, N, d, bf16, kBlockN) != FA_OK)
+    return FA_ERR_CUDA;
+  FwdParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.N = N;
+  p.bh = bh;
+  p.n_kv = (N + kBlockN - 1) / kBlockN;
+  p.n_pairs = (N + 2 * kBlockM - 1) / (2 * kBlockM);
+  p.n_units = bh * p.n_pairs;
+  p.scale_log2 = scale * kLog2e;
+  p.wait_limit_ns = wait_limit_ns();
+  p.debug_flags = g_debug_flags.load();
+  if (!(p.status = status_ptr())) return FA_ERR_CUDA;
+  const int grid = p.n_units < di.sms ? p.n_units : di.sms;
+  cudaError_t e = launch_fwd(d, bf16, causal != 0, tq, tk, tv, p, grid, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (check_common(B, H, N, d, 1.0f, FA_BF16) != FA_OK) return 0;
+  const size_t n_pad = ((size_t)N + kBlockN - 1) / kBlockN * kBlockN;
+  const size_t bh = (size_t)B * H;
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  return up(bh * n_pad * d * sizeof(float)) + 2 * up(bh * n_pad * sizeof(float));
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+           void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+           float scale, int causal, int dtype, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  int st = check_common(B, H, N, d, scale, dtype);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_MISALIGNED;
+  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_MISALIGNED;
+  DeviceInfo di;
+  if ((st = device_info(&di)) != FA_OK) return st;
+  const bool bf16 = dtype == FA_BF16;
+  const int bh = B * H;
+  BwdParams p{};
+  p.o = o;
+  p.dout = dout;
+  p.lse = lse;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.N = N;
+  p.n_kv = (N + kBlockN - 1) / kBlockN;
+  p.n_pad = p.n_kv * kBlockN;
+  p.bh = bh;
+  p.n_units = bh * p.n_kv;
+  p.scale = scale;
+  p.scale_log2 = scale * kLog2e;
+  p.wait_limit_ns = wait_limit_ns();
+  if (!(p.status = status_ptr())) return FA_ERR_CUDA;
+  const size_t acc_bytes = ((size_t)bh * p.n_pad * d * sizeof(float) + 255) / 256 * 256;
+  const size_t vec_bytes = ((size_t)bh * p.n_pad * sizeof(float) + 255) / 256 * 256;
+  p.dq_acc = static_cast<float*>(workspace);
+  p.dvec = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + acc_bytes);
+  p.lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + acc_bytes + vec_bytes);
+  CUtensorMap tq, tk, tv, tdo;
+  const int q_rows = (d == 64) ? 128 : 64;  // backward query tile (see fa_bwd_sm100.cu)
+  if (encode_tile_map(&tq, q, bh, N, d, bf16, q_rows) != FA_OK ||
+      encode_tile_map(&tk, k, bh, N, d, bf16, kBlockN) != FA_OK ||
+      encode_tile_map(&tv, v, bh, N, d, bf16, kBlockN) != FA_OK ||
+      encode_tile_map(&tdo, dout, bh, N, d, bf16, q_rows) != FA_OK)
+    return FA_ERR_CUDA;
+  const int grid = p.n_units < di.sms ? p.n_units : di.sms;
+  cudaError_t e = launch_bwd(d, bf16, causal != 0, tq, tk, tv, tdo, p, grid, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // extern "C"

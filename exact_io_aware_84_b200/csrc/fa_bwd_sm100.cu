@@ -1,0 +1,624 @@
+// Backward attention kernels for sm_100a.
+//
+// The backward recomputes P from Q, K and the forward's log-sum-exp instead
+// of storing it (marketmaker.cc "Backward pass: recompute instead of store").
+// With dP = dO V^T, D_i = sum_c dO_ic O_ic and dS = P o (dP - D):
+//   dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
+// Three launches:
+//   1. fa_bwd_prep:   D_i, LSE_i * log2(e) (+inf on padding rows), zero dQacc.
+//   2. fa_bwd_main:   one CTA per (batch*head, 128-key tile) unit, persistent;
+//                     loops over query tiles, keeps dK and dV in tensor memory,
+//                     adds each query tile's dQ into the fp32 accumulator with a
+//                     bulk shared->global reduce.
+//   3. fa_bwd_dq:     dQ = dtype(dQacc).
+//
+// fa_bwd_main works transposed (keys on the 128 tensor-memory lanes):
+//   S^T = K_j Q_i^T, dP^T = V_j dO_i^T            (SS MMAs, M = 128 keys)
+//   P^T = exp2(S^T * scale*log2e - LSE_i*log2e)    (softmax warpgroup)
+//   dS^T = P^T o (dP^T - D_i)                      (softmax warpgroup)
+//   dV += P^T dO_i, dK += dS^T Q_i                 (TS MMAs, A from TMEM)
+//   d = 64 : dQ_i   = dS K_j      (M = 128 queries, both operands MN-major)
+//   d = 128: dQ_i^T = K_j^T dS^T  (M = 128 head dims, both operands MN-major)
+// Query tile BR = 128 rows for d = 64 and 64 rows for d = 128, so that
+// S^T | dP^T | dV | dK | dQ fit in the 512 tensor-memory columns (448 used).
+// Roles (384 threads):
+//   warps 0-3   softmax warpgroup (thread = key = TMEM lane)
+//   warps 4-7   dQ / dK / dV epilogue warpgroup
+//   warp  8     TMA producer      warp 9   MMA issuer      warps 10-11 idle
+#include <cuda_fp16.h>
+
+#include "sm100_ptx.cuh"
+#include "fa_kernels.h"
+
+namespace fa {
+
+namespace {
+
+constexpr int kBwdThreads = 384;
+constexpr int kBProducerWarp = 8;
+constexpr int kBMmaWarp = 9;
+// Register split (same reasoning as the forward): every SM sub-partition holds
+// two warps of warpgroups 0-1 and one of warpgroup 2.
+constexpr int kBLaunchRegs = 168;
+constexpr int kBRegsWide = 192;
+constexpr int kBRegsNarrow = 120;
+static_assert(2 * kBRegsWide + kBRegsNarrow <= 3 * kBLaunchRegs, "register split exceeds a sub-partition's pool");
+
+template <int D>
+struct BwdLayout {
+  static constexpr int BR = (D == 64) ? 128 : 64;  // query rows per tile
+  static constexpr int kKV = kBlockN * D * 2;      // K or V tile bytes
+  static constexpr int kQT = BR * D * 2;           // Q or dO tile bytes
+  static constexpr int kDS = kBlockN * BR * 2;     // dS^T tile bytes
+  static constexpr int kStage = BR * D * 4;        // fp32 dQ staging bytes
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kKOff + kKV;
+  static constexpr int kQOff = kVOff + kKV;        // [2] stages
+  static constexpr int kDOOff = kQOff + 2 * kQT;   // [2] stages
+  static constexpr int kDSOff = kDOOff + 2 * kQT;
+  static constexpr int kStgOff = kDSOff + kDS;
+  static constexpr int kVecOff = kStgOff + kStage;  // [2] stages x (lse2[BR], dvec[BR])
+  static constexpr int kVecStage = 2 * BR * 4;
+  static constexpr int kBarOff = kVecOff + 2 * kVecStage;
+  // barriers
+  static constexpr int kKVFull = 0, kKVEmpty = 1;
+  static constexpr int kQFull = 2;   // [2]
+  static constexpr int kQEmpty = 4;  // [2]
+  static constexpr int kSFull = 6, kDPFull = 7, kPFull = 8, kDSFull = 9, kDSEmpty = 10;
+  static constexpr int kDQFull = 11, kDQEmpty = 12, kAccFull = 13, kAccEmpty = 14, kDrain = 15;
+  static constexpr int kNumBars = 16;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+  // tensor-memory columns
+  static constexpr uint32_t kColS = 0;
+  static constexpr uint32_t kColDP = BR;
+  static constexpr uint32_t kColDV = 2 * BR;
+  static constexpr uint32_t kColDK = 2 * BR + D;
+  static constexpr uint32_t kColDQ = 2 * BR + 2 * D;
+  static_assert(kColDQ + (D == 64 ? D : BR) <= 512, "tensor memory overflow");
+  static_assert(kAlloc <= 232448, "shared memory overflow");
+};
+
+struct BUnit {
+  int bh, jk, i0, i1;  // key tile jk; query tiles i0..i1 (inclusive)
+};
+
+template <int D, bool CAUSAL>
+__device__ __forceinline__ BUnit decode_bunit(int u, const BwdParams& p) {
+  constexpr int BR = BwdLayout<D>::BR;
+  BUnit r;
+  if (CAUSAL) {  // key tile 0 has the most query tiles: longest first
+    r.jk = u / p.bh;
+    r.bh = u % p.bh;
+  } else {       // neighbouring CTAs share a head (Q / dO reuse in L2)
+    r.jk = u % p.n_kv;
+    r.bh = u / p.n_kv;
+  }
+  r.i0 = CAUSAL ? (r.jk * kBlockN) / BR : 0;
+  r.i1 = (p.N + BR - 1) / BR - 1;
+  return r;
+}
+
+// Tile of R rows x D columns stored as D/64 column blocks of R x 128 B (SW128).
+// K-major operand view: advance 16 elements (32 B) per K step.
+template <int R>
+__device__ __forceinline__ uint64_t kmaj(uint32_t tile, int kstep) {
+  return make_sdesc_sw128(tile + (uint32_t)(kstep >> 2) * (R * 128) + (uint32_t)(kstep & 3) * 32, 16, 1024);
+}
+// MN-major operand view of the same storage (MN = the 64-wide column axis,
+// K = the row axis): column blocks R*128 bytes apart, 16 rows per K step.
+template <int R>
+__device__ __forceinline__ uint64_t mnmaj(uint32_t tile, int kstep) {
+  return make_sdesc_sw128(tile + (uint32_t)kstep * 2048, R * 128, 1024);
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(dst)),
+               "r"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+template <int D, bool BF16, bool CAUSAL>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    fa_bwd_main(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                const BwdParams p) {
+  using L = BwdLayout<D>;
+  constexpr int BR = L::BR;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t bars = base + L::kBarOff;
+  auto BAR = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::kMiscOff + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(L::kKVFull), 1);
+    mbar_init(BAR(L::kKVEmpty), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR(L::kQFull + s), 1);
+      mbar_init(BAR(L::kQEmpty + s), 1);
+    }
+    mbar_init(BAR(L::kSFull), 1);
+    mbar_init(BAR(L::kDPFull), 1);
+    mbar_init(BAR(L::kPFull), 128);
+    mbar_init(BAR(L::kDSFull), 128);
+    mbar_init(BAR(L::kDSEmpty), 1);
+    mbar_init(BAR(L::kDQFull), 1);
+    mbar_init(BAR(L::kDQEmpty), 128);
+    mbar_init(BAR(L::kAccFull), 1);
+    mbar_init(BAR(L::kAccEmpty), 128);
+    mbar_init(BAR(L::kDrain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kBProducerWarp) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{p.wait_limit_ns, abort_flag, p.status};
+  if (warp >= 8) regs_dec<kBRegsNarrow>();
+  else regs_inc<kBRegsWide>();
+
+  if (warp == kBProducerWarp) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      const uint64_t pol_kv = l2_policy_evict_first();
+      const uint64_t pol_q = l2_policy_evict_last();
+      uint32_t unit_iter = 0, q_iter = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
+        const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
+        if (unit_iter > 0 && !mbar_wait(BAR(L::kKVEmpty), (unit_iter - 1) & 1, wc)) { ok = false; break; }
+        mbar_arrive_expect_tx(BAR(L::kKVFull), 2 * L::kKV);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(base + L::kKOff + c * (kBlockN * 128), &tmK, BAR(L::kKVFull), c * 64, bu.jk * kBlockN, bu.bh, pol_kv);
+          tma_load_3d(base + L::kVOff + c * (kBlockN * 128), &tmV, BAR(L::kKVFull), c * 64, bu.jk * kBlockN, bu.bh, pol_kv);
+        }
+        for (int i = bu.i0; i <= bu.i1; ++i, ++q_iter) {
+          const uint32_t st = q_iter & 1, use = q_iter >> 1;
+          if (use > 0 && !mbar_wait(BAR(L::kQEmpty + st), (use - 1) & 1, wc)) { ok = false; break; }
+          const uint32_t fb = BAR(L::kQFull + st);
+          mbar_arrive_expect_tx(fb, 2 * L::kQT + L::kVecStage);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_3d(base + L::kQOff + st * L::kQT + c * (BR * 128), &tmQ, fb, c * 64, i * BR, bu.bh, pol_q);
+            tma_load_3d(base + L::kDOOff + st * L::kQT + c * (BR * 128), &tmDO, fb, c * 64, i * BR, bu.bh, pol_q);
+          }
+          const size_t row0 = (size_t)bu.bh * p.n_pad + (size_t)i * BR;
+          bulk_load(base + L::kVecOff + st * L::kVecStage, p.lse2 + row0, BR * 4, fb);
+          bulk_load(base + L::kVecOff + st * L::kVecStage + BR * 4, p.dvec + row0, BR * 4, fb);
+        }
+      }
+      if (!ok) {
+        if (unit_iter > 0) mbar_wait_drain(BAR(L::kKVFull), (unit_iter - 1) & 1, p.wait_limit_ns);
+        for (uint32_t s = 0; s < 2; ++s) {
+          const uint32_t issued = q_iter / 2 + (s < (q_iter & 1) ? 1u : 0u);
+          if (issued > 0) mbar_wait_drain(BAR(L::kQFull + s), (issued - 1) & 1, p.wait_limit_ns);
+        }
+      }
+    }
+  } else if (warp == kBMmaWarp) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = make_idesc_f16(BF16, kBlockN, BR, false, false);   // S^T, dP^T
+      constexpr uint32_t idesc_acc = make_idesc_f16(BF16, kBlockN, D, false, true);   // dV, dK
+      // dQ (d=64: M=128 queries, N=64) or dQ^T (d=128: M=128 dims, N=64 queries)
+      constexpr uint32_t idesc_dq = make_idesc_f16(BF16, 128, 64, true, true);
+      uint32_t unit_iter = 0, q_iter = 0, p_cnt = 0, ds_cnt = 0, dq_cnt = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
+        const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
+        if (!mbar_wait(BAR(L::kKVFull), unit_iter & 1, wc)) { ok = false; break; }
+        const uint32_t sK = base + L::kKOff, sV = base + L::kVOff;
+        // S^T for the first query tile
+        {
+          const uint32_t st = q_iter & 1;
+          if (!mbar_wait(BAR(L::kQFull + st), (q_iter >> 1) & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sQ = base + L::kQOff + st * L::kQT;
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_ss(tmem + L::kColS, kmaj<kBlockN>(sK, ks), kmaj<BR>(sQ, ks), idesc_s, ks > 0);
+          tc_commit(BAR(L::kSFull));
+        }
+        for (int i = bu.i0; i <= bu.i1; ++i, ++q_iter) {
+          const uint32_t st = q_iter & 1;
+          const uint32_t sQ = base + L::kQOff + st * L::kQT;
+          const uint32_t sDO = base + L::kDOOff + st * L::kQT;
+          const uint32_t first = (i == bu.i0);
+          // dP^T = V_j dO_i^T   (the dP region's previous contents, dS^T of
+          // tile i-1, were consumed by dK(i-1), issued earlier)
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_ss(tmem + L::kColDP, kmaj<kBlockN>(sV, ks), kmaj<BR>(sDO, ks), idesc_s, ks > 0);
+          tc_commit(BAR(L::kDPFull));
+          // dV += P^T dO_i
+          if (!mbar_wait(BAR(L::kPFull), p_cnt & 1, wc)) { ok = false; break; }
+          ++p_cnt;
+          if (first && unit_iter > 0 && !mbar_wait(BAR(L::kAccEmpty), (unit_iter - 1) & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < BR / 16; ++ks)
+            mma_ts(tmem + L::kColDV, tmem + L::kColS + 8u * ks, mnmaj<BR>(sDO, ks), idesc_acc, (!first || ks > 0) ? 1u : 0u);
+          // S^T for the next query tile (the S region's P^T was consumed by dV above)
+          if (i < bu.i1) {
+            const uint32_t st1 = (q_iter + 1) & 1;
+            if (!mbar_wait(BAR(L::kQFull + st1), ((q_iter + 1) >> 1) & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sQ1 = base + L::kQOff + st1 * L::kQT;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks)
+              mma_ss(tmem + L::kColS, kmaj<kBlockN>(sK, ks), kmaj<BR>(sQ1, ks), idesc_s, ks > 0);
+            tc_commit(BAR(L::kSFull));
+          }
+          // dK += dS^T Q_i
+          if (!mbar_wait(BAR(L::kDSFull), ds_cnt & 1, wc)) { ok = false; break; }
+          ++ds_cnt;
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < BR / 16; ++ks)
+            mma_ts(tmem + L::kColDK, tmem + L::kColDP + 8u * ks, mnmaj<BR>(sQ, ks), idesc_acc, (!first || ks > 0) ? 1u : 0u);
+          // dQ_i (d=64) or dQ_i^T (d=128) from dS^T in shared memory
+          if (dq_cnt > 0 && !mbar_wait(BAR(L::kDQEmpty), (dq_cnt - 1) & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sDS = base + L::kDSOff;
+#pragma unroll
+          for (int ks = 0; ks < kBlockN / 16; ++ks) {
+            if (D == 64)
+              mma_ss(tmem + L::kColDQ, mnmaj<kBlockN>(sDS, ks), mnmaj<kBlockN>(sK, ks), idesc_dq, ks > 0);
+            else
+              mma_ss(tmem + L::kColDQ, mnmaj<kBlockN>(sK, ks), mnmaj<kBlockN>(sDS, ks), idesc_dq, ks > 0);
+          }
+          tc_commit(BAR(L::kDQFull));
+          ++dq_cnt;
+          tc_commit(BAR(L::kQEmpty + st));   // Q_i, dO_i, LSE_i, D_i no longer read
+          tc_commit(BAR(L::kDSEmpty));       // dS^T shared tile no longer read
+        }
+        if (!ok) break;
+        tc_commit(BAR(L::kAccFull));
+        tc_commit(BAR(L::kKVEmpty));
+      }
+      tc_commit(BAR(L::kDrain));
+      mbar_wait_drain(BAR(L::kDrain), 0, p.wait_limit_ns);
+    }
+  } else if (warp < 4) {
+    // ---------------------------------------------------------------- softmax
+    const int key_in = threadIdx.x;  // 0..127 = TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + L::kColS;
+    const uint32_t tDP = tmem + lane_off + L::kColDP;
+    const float sl2 = p.scale_log2;
+    uint32_t q_iter = 0, s_cnt = 0, dp_cnt = 0, ds_cnt = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
+      const int key = bu.jk * kBlockN + key_in;
+      const bool key_ok = key < p.N;
+      for (int i = bu.i0; i <= bu.i1; ++i, ++q_iter) {
+        const uint32_t st = q_iter & 1;
+        if (!mbar_wait(BAR(L::kQFull + st), (q_iter >> 1) & 1, wc)) { ok = false; break; }
+        const float* lse2 = reinterpret_cast<const float*>(gbase + L::kVecOff + st * L::kVecStage);
+        const float* dvec = lse2 + BR;
+        if (!mbar_wait(BAR(L::kSFull), s_cnt & 1, wc)) { ok = false; break; }
+        ++s_cnt;
+        tc_fence_after();
+        const int q0 = i * BR;
+        // P^T = exp2(S^T * scale*log2e - LSE*log2e), masked; kept packed
+        uint32_t pk[BR / 2];
+#pragma unroll
+        for (int c = 0; c < BR / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tS + 32u * c, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int qa = 32 * c + 2 * e;
+            float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * e]), sl2, -lse2[qa]));
+            float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * e + 1]), sl2, -lse2[qa + 1]));
+            if (!key_ok || (CAUSAL && key > q0 + qa)) p0 = 0.f;
+            if (!key_ok || (CAUSAL && key > q0 + qa + 1)) p1 = 0.f;
+            pk[16 * c + e] = pack2<BF16>(p0, p1);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < BR / 32; ++c) tmem_st16(tS + 16u * c, pk + 16 * c);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR(L::kPFull));
+        // dS^T = P^T o (dP^T - D)
+        if (!mbar_wait(BAR(L::kDPFull), dp_cnt & 1, wc)) { ok = false; break; }
+        ++dp_cnt;
+        tc_fence_after();
+        if (ds_cnt > 0 && !mbar_wait(BAR(L::kDSEmpty), (ds_cnt - 1) & 1, wc)) { ok = false; break; }
+        ++ds_cnt;
+        uint32_t dsk[BR / 2];
+#pragma unroll
+        for (int c = 0; c < BR / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tDP + 32u * c, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int qa = 32 * c + 2 * e;
+            const uint32_t pp = pk[16 * c + e];
+            float p0, p1;
+            if constexpr (BF16) {
+              p0 = __uint_as_float(pp << 16);
+              p1 = __uint_as_float(pp & 0xFFFF0000u);
+            } else {
+              const __half2 h = *reinterpret_cast<const __half2*>(&pp);
+              p0 = __low2float(h);
+              p1 = __high2float(h);
+            }
+            const float ds0 = p0 * (__uint_as_float(r[2 * e]) - dvec[qa]);
+            const float ds1 = p1 * (__uint_as_float(r[2 * e + 1]) - dvec[qa + 1]);
+            dsk[16 * c + e] = pack2<BF16>(ds0, ds1);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < BR / 32; ++c) tmem_st16(tDP + 16u * c, dsk + 16 * c);
+        // dS^T row (this key) into the SW128 shared tile [key][query]:
+        // column block cb holds queries 64cb..64cb+63; 16-byte chunk ch of
+        // row `key_in` lives at chunk position ch ^ (key_in & 7).
+        uint8_t* ds_tile = gbase + L::kDSOff;
+#pragma unroll
+        for (int cb = 0; cb < BR / 64; ++cb) {
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            uint4 val = make_uint4(dsk[32 * cb + 4 * ch], dsk[32 * cb + 4 * ch + 1], dsk[32 * cb + 4 * ch + 2],
+                                   dsk[32 * cb + 4 * ch + 3]);
+            *reinterpret_cast<uint4*>(ds_tile + cb * (kBlockN * 128) + key_in * 128 + ((ch ^ (key_in & 7)) * 16)) = val;
+          }
+        }
+        tmem_wait_st();
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(BAR(L::kDSFull));
+      }
+    }
+  } else if (warp < 8) {
+    // ---------------------------------------------------------------- epilogue
+    const int t = threadIdx.x - 128;  // 0..127 = TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    float* stage = reinterpret_cast<float*>(gbase + L::kStgOff);
+    const uint32_t stage_s = base + L::kStgOff;
+    uint32_t dq_cnt = 0, unit_iter = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
+      const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
+      for (int i = bu.i0; i <= bu.i1; ++i) {
+        if (!mbar_wait(BAR(L::kDQFull), dq_cnt & 1, wc)) { ok = false; break; }
+        ++dq_cnt;
+        tc_fence_after();
+        // 64 fp32 columns per lane: d=64 -> lane = query, cols = dims;
+        //                           d=128 -> lane = dim, cols = queries.
+        uint32_t v[64];
+        tmem_ld32(tmem + lane_off + L::kColDQ, v);
+        tmem_ld32(tmem + lane_off + L::kColDQ + 32, v + 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(BAR(L::kDQEmpty));
+        // the previous bulk reduce must have finished reading the staging tile
+        if (t == 0) bulk_wait_read0();
+        named_bar_sync(1, 128);
+        if (D == 64) {
+          // row t of [128 queries][64 dims].  Lanes write different 16-byte
+          // chunks at the same time (chunk (e + t) mod 16 at step e) to spread
+          // shared-memory banks; the registers are first rotated by t chunks
+          // with a static barrel shifter so that no array is indexed by a
+          // lane-dependent value.
+          const int rot = t & 15;
+#pragma unroll
+          for (int b = 1; b < 16; b <<= 1) {
+            if (rot & b) {
+              uint32_t tmp[64];
+#pragma unroll
+              for (int e = 0; e < 64; ++e) tmp[e] = v[(e + 4 * b) & 63];
+#pragma unroll
+              for (int e = 0; e < 64; ++e) v[e] = tmp[e];
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int ch = (e + t) & 15;
+            float4 f = make_float4(__uint_as_float(v[4 * e]) * p.scale, __uint_as_float(v[4 * e + 1]) * p.scale,
+                                   __uint_as_float(v[4 * e + 2]) * p.scale, __uint_as_float(v[4 * e + 3]) * p.scale);
+            *reinterpret_cast<float4*>(stage + t * 64 + 4 * ch) = f;
+          }
+        } else {
+          // column t of [64 queries][128 dims]
+#pragma unroll
+          for (int q = 0; q < 64; ++q) stage[q * 128 + t] = __uint_as_float(v[q]) * p.scale;
+        }
+        fence_async_smem();
+        named_bar_sync(1, 128);
+        if (t == 0) {
+          bulk_reduce_add_f32(p.dq_acc + ((size_t)bu.bh * p.n_pad + (size_t)i * BR) * D, stage_s, L::kStage);
+          bulk_commit();
+        }
+      }
+      if (!ok) break;
+      // dK, dV of this key tile: lane = key
+      if (!mbar_wait(BAR(L::kAccFull), unit_iter & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      const int key = bu.jk * kBlockN + t;
+      const bool in_range = key < p.N;
+      const size_t rowoff = ((size_t)bu.bh * p.N + (size_t)(in_range ? key : 0)) * D * 2;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which ? L::kColDK : L::kColDV;
+        const float mul = which ? p.scale : 1.f;
+        uint8_t* dst = reinterpret_cast<uint8_t*>(which ? p.dk : p.dv) + rowoff;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_off + col + 32u * c, r);
+          tmem_wait_ld();
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack2<BF16>(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
+          if (in_range) {
+            uint4* o = reinterpret_cast<uint4*>(dst + c * 64);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(BAR(L::kAccEmpty));
+    }
+    if (t == 0) bulk_wait0();  // every dQ reduce has landed before the CTA exits
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kBProducerWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// D_i = sum_c dO_ic O_ic; lse2_i = LSE_i * log2(e); both +0 / +inf on the
+// padding rows N..n_pad-1; dQacc rows zeroed.  One warp per row.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_prep(const BwdParams p) {
+  const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int total = p.bh * p.n_pad;
+  if (warp_global >= total) return;
+  const int bh = warp_global / p.n_pad;
+  const int row = warp_global % p.n_pad;
+  float acc = 0.f;
+  if (row < p.N) {
+    const size_t off = ((size_t)bh * p.N + row) * D;
+    constexpr int PER = D / 32;  // elements per lane (2 or 4)
+    const uint8_t* o8 = reinterpret_cast<const uint8_t*>(p.o) + off * 2 + lane * PER * 2;
+    const uint8_t* d8 = reinterpret_cast<const uint8_t*>(p.dout) + off * 2 + lane * PER * 2;
+    uint32_t ow[PER / 2], dw[PER / 2];
+#pragma unroll
+    for (int e = 0; e < PER / 2; ++e) {
+      ow[e] = reinterpret_cast<const uint32_t*>(o8)[e];
+      dw[e] = reinterpret_cast<const uint32_t*>(d8)[e];
+    }
+#pragma unroll
+    for (int e = 0; e < PER / 2; ++e) {
+      float a0, a1, b0, b1;
+      if constexpr (BF16) {
+        a0 = __uint_as_float(ow[e] << 16);
+        a1 = __uint_as_float(ow[e] & 0xFFFF0000u);
+        b0 = __uint_as_float(dw[e] << 16);
+        b1 = __uint_as_float(dw[e] & 0xFFFF0000u);
+      } else {
+        const __half2 ha = *reinterpret_cast<const __half2*>(&ow[e]);
+        const __half2 hb = *reinterpret_cast<const __half2*>(&dw[e]);
+        a0 = __low2float(ha);
+        a1 = __high2float(ha);
+        b0 = __low2float(hb);
+        b1 = __high2float(hb);
+      }
+      acc = fmaf(a0, b0, acc);
+      acc = fmaf(a1, b1, acc);
+    }
+  }
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  const size_t prow = (size_t)bh * p.n_pad + row;
+  if (lane == 0) {
+    p.dvec[prow] = acc;
+    p.lse2[prow] = row < p.N ? p.lse[(size_t)bh * p.N + row] * 1.4426950408889634f : INFINITY;
+  }
+  float4* acc_row = reinterpret_cast<float4*>(p.dq_acc + prow * D);
+#pragma unroll
+  for (int e = lane; e < D / 4; e += 32) acc_row[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// dQ = dtype(dQacc) for the real rows.  One thread per 8 elements.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_dq(const BwdParams p) {
+  const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;  // 8-element group
+  const size_t groups = (size_t)p.bh * p.N * (D / 8);
+  if (idx >= groups) return;
+  const size_t row = idx / (D / 8);  // bh * N + n
+  const int g = (int)(idx % (D / 8));
+  const size_t bh = row / p.N, n = row % p.N;
+  const float4* src = reinterpret_cast<const float4*>(p.dq_acc + (bh * p.n_pad + n) * D + g * 8);
+  const float4 a = src[0], b = src[1];
+  uint4 w = make_uint4(pack2<BF16>(a.x, a.y), pack2<BF16>(a.z, a.w), pack2<BF16>(b.x, b.y), pack2<BF16>(b.z, b.w));
+  reinterpret_cast<uint4*>(p.dq)[idx] = w;
+}
+
+template <int D, bool BF16, bool CAUSAL>
+cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const CUtensorMap& tdo, const BwdParams& p, int grid, cudaStream_t st) {
+  {
+    const long long warps = (long long)p.bh * p.n_pad;
+    const int blocks = (int)((warps * 32 + 255) / 256);
+    fa_bwd_prep<D, BF16><<<blocks, 256, 0, st>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  {
+    auto kern = fa_bwd_main<D, BF16, CAUSAL>;
+    constexpr int smem = BwdLayout<D>::kAlloc;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kBwdThreads, smem, st>>>(tq, tk, tv, tdo, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  {
+    const long long groups = (long long)p.bh * p.N * (D / 8);
+    const int blocks = (int)((groups + 255) / 256);
+    fa_bwd_dq<D, BF16><<<blocks, 256, 0, st>>>(p);
+    return cudaGetLastError();
+  }
+}
+
+}  // namespace
+
+int bwd_threads() { return kBwdThreads; }
+
+cudaError_t launch_bwd(int d, bool bf16, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
+                       const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p, int grid,
+                       cudaStream_t st) {
+#define FA_BWD_CASE(DD, BB, CC) \
+  if (d == DD && bf16 == BB && causal == CC) return launch_bwd_t<DD, BB, CC>(tq, tk, tv, tdo, p, grid, st);
+  FA_BWD_CASE(64, true, false)
+  FA_BWD_CASE(64, true, true)
+  FA_BWD_CASE(64, false, false)
+  FA_BWD_CASE(64, false, true)
+  FA_BWD_CASE(128, true, false)
+  FA_BWD_CASE(128, true, true)
+  FA_BWD_CASE(128, false, false)
+  FA_BWD_CASE(128, false, true)
+#undef FA_BWD_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace fa

@@ -1,0 +1,423 @@
+// Forward attention kernel for sm_100a.
+//
+// O = softmax(scale * Q K^T [causal]) V and LSE, one head at a time, with the
+// online-softmax recurrence over 128-key tiles (marketmaker.cc "The Flash
+// Attention algorithm" / "Online softmax recurrence"; ultralytics.com
+// glossary "How Flash Attention works").  S and P live only in tensor memory.
+//
+// Work unit: one (batch*head, pair of 128-row query tiles).  Persistent CTAs
+// (one per SM) walk the units with a static stride; causal units are taken
+// longest first.  Roles inside a CTA (384 threads = 3 warpgroups):
+//   warps 0-3  softmax warpgroup for query tile 0 (thread = row = TMEM lane)
+//   warps 4-7  softmax warpgroup for query tile 1
+//   warp  8    TMA producer: Q tiles once per unit, K/V tiles through a ring
+//   warp  9    MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j
+//   warps 10-11 idle (they complete the third warpgroup, so that the register
+//              split below moves registers within every SM sub-partition)
+// Tensor memory (512 columns): S_0 | S_1 | O_0 | O_1.  P (16-bit) is written
+// over the first half of its S tile and consumed from there by the PV MMA.
+// The two query tiles alternate on the tensor core: while one softmax
+// warpgroup exponentiates its S tile, the MMAs of the other tile run.
+//
+// Rescaling is deferred and conditional: O and l keep a stale running max
+// until the max grows by more than 2^8; since O and l are scaled alike, the
+// final O / l is unchanged (exactness is kept; only the headroom is bounded).
+#include "sm100_ptx.cuh"
+#include "fa_kernels.h"
+
+namespace fa {
+
+namespace {
+
+constexpr int kFwdThreads = 384;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only if max grows > 2^8
+// Register split.  Launch: 384 threads x 168 registers.  Warp w runs on SM
+// sub-partition w % 4, which therefore holds warps {k, k+4, k+8}: two softmax
+// warps and one warp of the producer/MMA warpgroup.  Each sub-partition's
+// share after the split must not exceed its launch share (3 x 168).
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsSoftmax = 224;
+constexpr int kRegsOther = 56;
+static_assert(2 * kRegsSoftmax + kRegsOther <= 3 * kLaunchRegs, "register split exceeds a sub-partition's pool");
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kTile = kBlockM * D * 2;  // bytes of one 128 x D 16-bit tile
+  static constexpr int kSlots = (D == 128) ? 4 : 8;
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = 2 * kTile;
+  static constexpr int kBarOff = kKVOff + kSlots * kTile;
+  // barrier indices
+  static constexpr int kQFull = 0;
+  static constexpr int kQEmpty = 1;
+  static constexpr int kKVFull = 2;
+  static constexpr int kKVEmpty = 2 + kSlots;
+  static constexpr int kSFull = 2 + 2 * kSlots;  // [2]
+  static constexpr int kPFull = kSFull + 2;      // [2]
+  static constexpr int kOFull = kPFull + 2;      // [2]
+  static constexpr int kOEmpty = kOFull + 2;     // [2]
+  static constexpr int kDrain = kOEmpty + 2;
+  static constexpr int kNumBars = kDrain + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B
+  // tensor-memory columns
+  static constexpr uint32_t kColS0 = 0;
+  static constexpr uint32_t kColO0 = 256;
+};
+
+struct UnitInfo {
+  int bh;
+  int r0_0, r0_1;  // first row of query tile 0 / 1
+  int nb_0, nb_1;  // key/value tiles each query tile visits (0 = tile absent)
+  int nmax;
+  __device__ __forceinline__ int r0(int t) const { return t ? r0_1 : r0_0; }
+  __device__ __forceinline__ int nb(int t) const { return t ? nb_1 : nb_0; }
+};
+
+template <bool CAUSAL>
+__device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams& p) {
+  UnitInfo ui;
+  int pair;
+  if (CAUSAL) {  // longest units first
+    pair = p.n_pairs - 1 - u / p.bh;
+    ui.bh = u % p.bh;
+  } else {       // neighbouring CTAs share a head (K/V reuse in L2)
+    pair = u % p.n_pairs;
+    ui.bh = u / p.n_pairs;
+  }
+  ui.r0_0 = pair * 2 * kBlockM;
+  ui.r0_1 = ui.r0_0 + kBlockM;
+  ui.nb_0 = CAUSAL ? (ui.r0_0 / kBlockN + 1) : p.n_kv;  // tile 0 always exists
+  ui.nb_1 = ui.r0_1 < p.N ? (CAUSAL ? (ui.r0_1 / kBlockN + 1) : p.n_kv) : 0;
+  ui.nmax = ui.nb_1 > ui.nb_0 ? ui.nb_1 : ui.nb_0;
+  return ui;
+}
+
+// K-major SW128 operand (Q tile or K tile): rows of 64 elements (128 B);
+// a D-wide tile is stored as D/64 column blocks of 128 rows x 128 B.
+template <int D>
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kstep) {
+  const uint32_t addr = tile + (uint32_t)(kstep >> 2) * (kBlockM * 128) + (uint32_t)(kstep & 3) * 32;
+  return make_sdesc_sw128(addr, 16, 1024);
+}
+
+// V tile as the MN-major B operand of O += P V: N = head dim (contiguous),
+// K = key index.  Column blocks of 64 are kBlockN*128 bytes apart (LBO),
+// 8-key groups 1024 bytes apart (SBO); one 16-key K step = 2048 bytes.
+__device__ __forceinline__ uint64_t v_desc(uint32_t tile, int kstep) {
+  return make_sdesc_sw128(tile + (uint32_t)kstep * 2048, kBlockN * 128, 1024);
+}
+
+template <int D, bool BF16, bool CAUSAL>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using L = FwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t bars = base + L::kBarOff;
+  auto BAR = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::kMiscOff + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(L::kQFull), 1);
+    mbar_init(BAR(L::kQEmpty), 1);
+    for (int s = 0; s < L::kSlots; ++s) {
+      mbar_init(BAR(L::kKVFull + s), 1);
+      mbar_init(BAR(L::kKVEmpty + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(BAR(L::kSFull + t), 1);
+      mbar_init(BAR(L::kPFull + t), 128);
+      mbar_init(BAR(L::kOFull + t), 1);
+      mbar_init(BAR(L::kOEmpty + t), 128);
+    }
+    mbar_init(BAR(L::kDrain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kProducerWarp) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{p.wait_limit_ns, abort_flag, p.status};
+
+  if (warp >= 8) regs_dec<kRegsOther>();
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const uint64_t pol_kv = l2_policy_evict_last();
+      const uint64_t pol_q = l2_policy_evict_first();
+      uint32_t kv_iter = 0, unit_iter = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
+        const UnitInfo ui = decode_unit<CAUSAL>(u, p);
+        if (unit_iter > 0 && !mbar_wait(BAR(L::kQEmpty), (unit_iter - 1) & 1, wc)) { ok = false; break; }
+        const uint32_t qbytes = (ui.nb_1 > 0 ? 2u : 1u) * L::kTile;
+        mbar_arrive_expect_tx(BAR(L::kQFull), qbytes);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (ui.nb(t) == 0) continue;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(base + L::kQOff + t * L::kTile + c * (kBlockM * 128), &tmQ, BAR(L::kQFull), c * 64,
+                        ui.r0(t), ui.bh, pol_q);
+        }
+        for (int j = 0; j < ui.nmax && ok; ++j) {
+          for (int kv = 0; kv < 2; ++kv, ++kv_iter) {
+            const uint32_t slot = kv_iter % L::kSlots;
+            const uint32_t use = kv_iter / L::kSlots;
+            if (use > 0 && !mbar_wait(BAR(L::kKVEmpty + slot), (use - 1) & 1, wc)) { ok = false; break; }
+            mbar_arrive_expect_tx(BAR(L::kKVFull + slot), L::kTile);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(base + L::kKVOff + slot * L::kTile + c * (kBlockN * 128), kv ? &tmV : &tmK,
+                          BAR(L::kKVFull + slot), c * 64, j * kBlockN, ui.bh, pol_kv);
+          }
+        }
+      }
+      if (!ok) {
+        // Let every copy already issued land before the CTA exits.
+        for (uint32_t s = 0; s < (uint32_t)L::kSlots; ++s) {
+          const uint32_t issued = kv_iter / L::kSlots + (s < kv_iter % L::kSlots ? 1u : 0u);
+          if (issued > 0) mbar_wait_drain(BAR(L::kKVFull + s), (issued - 1) & 1, p.wait_limit_ns);
+        }
+        if (unit_iter > 0) mbar_wait_drain(BAR(L::kQFull), (unit_iter - 1) & 1, p.wait_limit_ns);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = make_idesc_f16(BF16, kBlockM, kBlockN, false, false);
+      constexpr uint32_t idesc_pv = make_idesc_f16(BF16, kBlockM, D, false, true);
+      uint32_t kv_iter = 0, unit_iter = 0;
+      uint32_t p_cnt0 = 0, p_cnt1 = 0, o_uses0 = 0, o_uses1 = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
+        const UnitInfo ui = decode_unit<CAUSAL>(u, p);
+        if (!mbar_wait(BAR(L::kQFull), unit_iter & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kv_base = kv_iter;
+        for (int j = 0; j <= ui.nmax && ok; ++j) {
+          const uint32_t k_idx = kv_base + 2 * j, v_idx = kv_base + 2 * (j - 1) + 1;
+          if (j < ui.nmax) {
+            if (!mbar_wait(BAR(L::kKVFull + k_idx % L::kSlots), (k_idx / L::kSlots) & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+          }
+          bool v_ready = false;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const int nbt = ui.nb(t);
+            if (!ok || nbt == 0) continue;
+            const uint32_t colS = L::kColS0 + 128u * t;
+            const uint32_t colO = L::kColO0 + (uint32_t)D * t;
+            const uint32_t pc = t ? p_cnt1 : p_cnt0;
+            const uint32_t ou = t ? o_uses1 : o_uses0;
+            if (j >= 1 && j <= nbt) {
+              // O_t (+)= P_t V_{j-1}
+              ok = mbar_wait(BAR(L::kPFull + t), pc & 1, wc);
+              if (t) ++p_cnt1; else ++p_cnt0;
+              if (ok && j == 1 && ou > 0) ok = mbar_wait(BAR(L::kOEmpty + t), (ou - 1) & 1, wc);
+              if (ok && !v_ready) {
+                ok = mbar_wait(BAR(L::kKVFull + v_idx % L::kSlots), (v_idx / L::kSlots) & 1, wc);
+                v_ready = true;
+              }
+              if (!ok) continue;
+              tc_fence_after();
+              const uint32_t vt = base + L::kKVOff + (v_idx % L::kSlots) * L::kTile;
+#pragma unroll
+              for (int ks = 0; ks < kBlockN / 16; ++ks)
+                mma_ts(tmem + colO, tmem + colS + 8u * ks, v_desc(vt, ks), idesc_pv, (j > 1 || ks > 0) ? 1u : 0u);
+              if (j == nbt) tc_commit(BAR(L::kOFull + t));
+            }
+            if (j < nbt) {
+              // S_t = Q_t K_j^T
+              const uint32_t qt = base + L::kQOff + t * L::kTile;
+              const uint32_t kt = base + L::kKVOff + (k_idx % L::kSlots) * L::kTile;
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks)
+                mma_ss(tmem + colS, kmajor_desc<D>(qt, ks), kmajor_desc<D>(kt, ks), idesc_s, ks > 0 ? 1u : 0u);
+              tc_commit(BAR(L::kSFull + t));
+            }
+          }
+          if (!ok) break;
+          if (j == ui.nmax - 1) tc_commit(BAR(L::kQEmpty));
+          if (j >= 1) {
+            tc_commit(BAR(L::kKVEmpty + (kv_base + 2 * (j - 1)) % L::kSlots));
+            tc_commit(BAR(L::kKVEmpty + v_idx % L::kSlots));
+          }
+        }
+        kv_iter = kv_base + 2 * ui.nmax;
+        o_uses0 += 1;
+        o_uses1 += ui.nb_1 > 0 ? 1u : 0u;
+      }
+      // Make sure no MMA is still reading shared memory or writing tensor
+      // memory when the CTA leaves (normal exit: they are all done already).
+      tc_commit(BAR(L::kDrain));
+      mbar_wait_drain(BAR(L::kDrain), 0, p.wait_limit_ns);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax
+    regs_inc<kRegsSoftmax>();
+    const int t = warp >> 2;                       // query tile of this warpgroup
+    const int r_in = threadIdx.x & 127;            // row within the tile = TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + L::kColS0 + 128u * t;
+    const uint32_t tO = tmem + lane_off + L::kColO0 + (uint32_t)D * t;
+    const float sl2 = p.scale_log2;
+    uint32_t s_cnt = 0, o_cnt = 0;
+    int unit_iter = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
+      const UnitInfo ui = decode_unit<CAUSAL>(u, p);
+      const int nb = ui.nb(t);
+      if (nb == 0) continue;
+      const int row = ui.r0(t) + r_in;
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < nb; ++j) {
+        if (!mbar_wait(BAR(L::kSFull + t), s_cnt & 1, wc)) { ok = false; break; }
+        ++s_cnt;
+        tc_fence_after();
+        uint32_t sr[kBlockN];
+#pragma unroll
+        for (int c = 0; c < kBlockN / 32; ++c) tmem_ld32(tS + 32u * c, sr + 32 * c);
+        tmem_wait_ld();
+        float s[kBlockN];
+#pragma unroll
+        for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(sr[c]);
+        const int kbase = j * kBlockN;
+        if (CAUSAL && j == nb - 1) {
+#pragma unroll
+          for (int c = 0; c < kBlockN; ++c)
+            if (kbase + c > row) s[c] = -INFINITY;
+        } else if (!CAUSAL && kbase + kBlockN > p.N) {
+#pragma unroll
+          for (int c = 0; c < kBlockN; ++c)
+            if (kbase + c >= p.N) s[c] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int c = 1; c < kBlockN; ++c) mx = fmaxf(mx, s[c]);
+        const float m_new = fmaxf(m_run, mx * sl2);
+        if (j == 0) {
+          m_run = (m_new == -INFINITY) ? 0.f : m_new;
+        } else if (m_new > m_run + kRescaleThreshold) {
+          const float alpha = ex2_approx(m_run - m_new);
+          l_run *= alpha;
+          m_run = m_new;
+          // O_t was last written by PV of tile j-1, which completed before
+          // S_j was signalled (tcgen05 ops of one thread complete in order).
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32u * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + 32u * c, o);
+          }
+        }
+        const float neg_m = -m_run;
+        float sum = 0.f;
+#pragma unroll
+        for (int q = 0; q < kBlockN / 32; ++q) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2_approx(fmaf(s[32 * q + 2 * e], sl2, neg_m));
+            const float p1 = ex2_approx(fmaf(s[32 * q + 2 * e + 1], sl2, neg_m));
+            sum += p0 + p1;
+            pk[e] = pack2<BF16>(p0, p1);
+          }
+          tmem_st16(tS + 16u * q, pk);
+        }
+        l_run += sum;
+        tmem_wait_st();
+        tc_fence_before();
+        const bool withhold = (p.debug_flags & 1) && unit_iter == 0 && j == 0 && t == 0;
+        if (!withhold) mbar_arrive(BAR(L::kPFull + t));
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l -> dtype -> global; LSE = (m + log2 l) ln 2
+      if (!mbar_wait(BAR(L::kOFull + t), o_cnt & 1, wc)) { ok = false; break; }
+      ++o_cnt;
+      tc_fence_after();
+      const float inv_l = 1.f / l_run;
+      const bool in_range = row < p.N;
+      uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + ((size_t)ui.bh * p.N + (size_t)(in_range ? row : 0)) * D * 2;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32u * c, o);
+        tmem_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack2<BF16>(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+        if (in_range) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(BAR(L::kOEmpty + t));
+      if (in_range) p.lse[(size_t)ui.bh * p.N + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kProducerWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, bool BF16, bool CAUSAL>
+cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const FwdParams& p, int grid, cudaStream_t st) {
+  auto kern = fa_fwd_kernel<D, BF16, CAUSAL>;
+  constexpr int smem = FwdLayout<D>::kAlloc;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kFwdThreads, smem, st>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int fwd_threads() { return kFwdThreads; }
+
+cudaError_t launch_fwd(int d, bool bf16, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
+                       const CUtensorMap& tv, const FwdParams& p, int grid, cudaStream_t st) {
+#define FA_FWD_CASE(DD, BB, CC) \
+  if (d == DD && bf16 == BB && causal == CC) return launch_fwd_t<DD, BB, CC>(tq, tk, tv, p, grid, st);
+  FA_FWD_CASE(64, true, false)
+  FA_FWD_CASE(64, true, true)
+  FA_FWD_CASE(64, false, false)
+  FA_FWD_CASE(64, false, true)
+  FA_FWD_CASE(128, true, false)
+  FA_FWD_CASE(128, true, true)
+  FA_FWD_CASE(128, false, false)
+  FA_FWD_CASE(128, false, true)
+#undef FA_FWD_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace fa

@@ -1,0 +1,60 @@
+// Parameter blocks and launch entry points shared by the C-ABI front end
+// (fa_api.cu) and the kernel translation units.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace fa {
+
+constexpr int kBlockM = 128;  // query rows per Q tile (tcgen05 M)
+constexpr int kBlockN = 128;  // keys per K/V tile
+
+struct FwdParams {
+  void* o;             // [B*H, N, D] dtype
+  float* lse;          // [B*H, N] fp32
+  int N;               // sequence length
+  int bh;              // B*H
+  int n_kv;            // ceil(N / 128): key/value tiles per head
+  int n_pairs;         // ceil(N / 256): pairs of 128-row Q tiles per head
+  int n_units;         // bh * n_pairs
+  float scale_log2;    // scale * log2(e)
+  uint64_t wait_limit_ns;
+  int* status;         // device status word
+  int debug_flags;
+};
+
+struct BwdParams {
+  const void* o;       // forward output, [B*H, N, D]
+  const void* dout;    // dO, [B*H, N, D]
+  const float* lse;    // [B*H, N]
+  void* dq;            // [B*H, N, D]
+  void* dk;            // [B*H, N, D]
+  void* dv;            // [B*H, N, D]
+  float* dq_acc;       // [B*H, n_pad, D] fp32 workspace
+  float* dvec;         // [B*H, n_pad] fp32 workspace (D_i)
+  float* lse2;         // [B*H, n_pad] fp32 workspace (LSE_i * log2 e; +inf on padding)
+  int N;
+  int n_pad;           // ceil(N / 128) * 128
+  int bh;
+  int n_kv;            // ceil(N / 128)
+  int n_units;         // bh * n_kv
+  float scale;         // softmax scale
+  float scale_log2;    // scale * log2(e)
+  uint64_t wait_limit_ns;
+  int* status;         // device status word
+};
+
+// Launchers (return cudaError_t of the launch).
+cudaError_t launch_fwd(int d, bool bf16, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
+                       const CUtensorMap& tv, const FwdParams& p, int grid, cudaStream_t st);
+
+cudaError_t launch_bwd(int d, bool bf16, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
+                       const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p, int grid,
+                       cudaStream_t st);
+
+int fwd_threads();
+int bwd_threads();
+
+}  // namespace fa

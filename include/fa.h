@@ -1,0 +1,138 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact, IO-aware scaled-dot-product attention
+ * (forward and backward) for NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  For every batch b and head h, with S = scale * Q K^T
+ * (entries with key j > query i set to -inf when `causal` is non-zero):
+ *     LSE_i = ln sum_j exp(S_ij),   P = exp(S - LSE),   O = P V.
+ * The N x N matrices S and P are never written to device memory: the forward
+ * streams key/value tiles through on-chip memory with the online-softmax
+ * recurrence and writes only O and the per-row log-sum-exp; the backward
+ * recomputes P from Q, K and the stored LSE.  Sources (page title, section):
+ *   - marketmaker.cc, "Flash Attention and the sequence-length problem":
+ *     "Why attention is memory-bound" (the definition), "The Flash Attention
+ *     algorithm" (tiling over query and key/value blocks), "Online softmax
+ *     recurrence", "Backward pass: recompute instead of store", "Causal
+ *     masking" (future tiles skipped), "Integration is eight lines" (the
+ *     (batch, heads, seq, head_dim) layout and the is_causal flag);
+ *   - ultralytics.com glossary "Flash Attention", "How Flash Attention works"
+ *     (only the output and two numbers per row go back to HBM).
+ * Results are exact in exact arithmetic, not bitwise: the fp32 accumulation
+ * order and the rounding of P to the input type differ from a two-pass
+ * evaluation (delect.ru glossary "FlashAttention", "What is confirmed").
+ *
+ * Layout.  q, k, v, o, dout, dq, dk, dv: [B, H, N, d] contiguous, row stride d
+ * elements, element type `dtype` (FA_BF16 or FA_FP16).  lse: [B, H, N]
+ * contiguous float32, natural log.  Every pointer is a device pointer
+ * aligned to 16 bytes.  Supported: d in {64, 128}; N >= 1 (any N: the last
+ * tile may be ragged); B >= 1, H >= 1; B*H*N*d < 2^31.
+ *
+ * Ownership.  The caller allocates and owns every buffer.  The library never
+ * allocates device memory and keeps no per-call state.  All calls are
+ * asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ * stream).  Outputs are overwritten, never accumulated into.
+ *
+ * Errors.  Every entry point returns an fa_status.  Argument errors are
+ * detected on the host before anything is launched.  A kernel whose internal
+ * pipeline wait exceeds the wait limit (default 1000 ms, see
+ * fa_debug_set_wait_limit_ms) abandons its work, records FA_ERR_TIMEOUT in a
+ * device status word and returns; fa_last_device_status() reports it.
+ * Nothing in the library traps or asserts on the device.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, size overflow */
+  FA_ERR_UNSUPPORTED = 2, /* head dim other than 64/128, unknown dtype */
+  FA_ERR_MISALIGNED = 3,  /* a pointer not 16-byte aligned */
+  FA_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
+  FA_ERR_TIMEOUT = 5,     /* a kernel gave up on a pipeline wait */
+  FA_ERR_WORKSPACE = 6,   /* workspace missing or smaller than required */
+  FA_ERR_NO_DEVICE = 7    /* no sm_100 device is current */
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
+
+/*
+ * Forward: O = softmax(scale * Q K^T [causal]) V and LSE.
+ *   q, k, v : inputs, [B,H,N,d], dtype.
+ *   o       : output, [B,H,N,d], dtype (round-to-nearest-even of O).
+ *   lse     : output, [B,H,N] float32, LSE_i = ln sum_j exp(S_ij).
+ *   scale   : score multiplier (1/sqrt(d) for standard attention).
+ *   causal  : non-zero => key j attends to query i only if j <= i
+ *             (top-left aligned; key blocks entirely in the future are
+ *             skipped).
+ * One kernel launch.  Source: marketmaker.cc "The Flash Attention
+ * algorithm" and "Online softmax recurrence"; ultralytics.com glossary
+ * "How Flash Attention works".
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+           float scale, int causal, int dtype, void* stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs for these sizes: a float32 dQ
+ * accumulator of B*H*ceil(N/128)*128*d elements, then two float32 row
+ * vectors of B*H*ceil(N/128)*128 elements (D_i = sum_c dO_ic O_ic, and
+ * LSE_i * log2(e)), each section rounded up to 256 bytes.  Returns 0 for
+ * invalid sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward: given dO = dL/dO, computes dQ, dK, dV by recomputing P from Q, K
+ * and the forward's LSE (never storing P):
+ *   D_i = sum_c dO_ic O_ic;  dV = P^T dO;  dP = dO V^T;  dS = P o (dP - D);
+ *   dQ = scale dS K;  dK = scale dS^T Q.
+ *   q, k, v, o, dout : inputs, [B,H,N,d], dtype (o is the forward's output).
+ *   lse              : input, [B,H,N] float32 from fa_fwd.
+ *   dq, dk, dv       : outputs, [B,H,N,d], dtype.
+ *   workspace        : device buffer of at least fa_bwd_workspace_size()
+ *                      bytes, 256-byte aligned; contents on entry ignored.
+ * Three kernel launches on `stream` (D and dQ-accumulator zeroing; dK/dV with
+ * dQ accumulation; dQ conversion).  Source: marketmaker.cc "Backward pass:
+ * recompute instead of store"; delect.ru glossary, the backward-recomputation
+ * claim.  The gradient formulas are the softmax Jacobian (the pages do not
+ * print them).
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+           void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+           float scale, int causal, int dtype, void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fa_status_string(int status);
+
+/*
+ * Synchronises `stream`, then returns FA_ERR_TIMEOUT if any kernel of this
+ * library on the current device gave up on a pipeline wait since the last
+ * call (FA_OK otherwise), and clears that record.  Returns FA_ERR_CUDA if
+ * the synchronisation itself fails.
+ */
+int fa_last_device_status(void* stream);
+
+/*
+ * Diagnostics.  fa_debug_set_wait_limit_ms sets the per-wait limit used by
+ * later launches (process-wide; ms >= 1).  fa_debug_set_flags sets
+ * process-wide debug flags: bit 0 makes the forward kernel withhold one
+ * pipeline arrival on its first tile, so that its bounded waits run out
+ * and the launch ends with FA_ERR_TIMEOUT (used by the timeout test);
+ * 0 restores normal operation.  Both return FA_OK or FA_ERR_INVALID_ARG.
+ */
+int fa_debug_set_wait_limit_ms(int ms);
+int fa_debug_set_flags(int flags);
+
+/* Version string of the library build. */
+const char* fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -1,0 +1,136 @@
+"""Forward parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small shapes span several 128-row tiles and ragged tails; the named
+workloads run at full size with every output computed on the GPU and rows
+sampled for the oracle where it cannot do all of them quickly.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import exact_io_aware_84_b200 as fa
+from exact_io_aware_84_b200.inputs import Workload, make_inputs, workload
+from oracle import attn_fwd_ref, attn_fwd_rows_ref
+from parity import check_o_lse, sample_rows, to64
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu(x):
+    return {k: v.cuda() for k, v in x.items()}
+
+
+def _run(w, x=None):
+    x = make_inputs(w, with_grad=False) if x is None else x
+    g = _gpu(x)
+    o, lse = fa.fa_fwd(g["q"], g["k"], g["v"], scale=w.scale, causal=w.causal)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == fa.FA_OK
+    return x, o, lse
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [1, 17, 128, 129, 255, 256, 257, 384, 513])
+def test_small_shapes_bf16(N, d, causal):
+    w = Workload("small", 2, 3, N, d, "bf16", causal, 1.0 / d ** 0.5, False, seed=N + d)
+    x, o, lse = _run(w)
+    o_ref, lse_ref = attn_fwd_ref(to64(x["q"]), to64(x["k"]), to64(x["v"]), w.scale, causal)
+    check_o_lse(to64(o), to64(lse), o_ref, lse_ref, f"N={N} d={d} causal={causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [200, 640])
+def test_small_shapes_fp16(N, d, causal):
+    w = Workload("small16", 1, 2, N, d, "fp16", causal, 1.0 / d ** 0.5, False, seed=7)
+    x, o, lse = _run(w)
+    o_ref, lse_ref = attn_fwd_ref(to64(x["q"]), to64(x["k"]), to64(x["v"]), w.scale, causal)
+    check_o_lse(to64(o), to64(lse), o_ref, lse_ref, f"fp16 N={N} d={d} causal={causal}")
+
+
+def test_many_units_per_cta():
+    # more (head, tile-pair) units than SMs: each persistent CTA runs several
+    w = Workload("many", 4, 40, 512, 64, "bf16", False, 0.125, False, seed=3)
+    x, o, lse = _run(w)
+    o_ref, lse_ref = attn_fwd_ref(to64(x["q"]), to64(x["k"]), to64(x["v"]), w.scale, False)
+    check_o_lse(to64(o), to64(lse), o_ref, lse_ref, "many units")
+
+
+def test_many_units_per_cta_causal_d128():
+    w = Workload("many_c", 2, 48, 640, 128, "bf16", True, 128 ** -0.5, False, seed=4)
+    x, o, lse = _run(w)
+    o_ref, lse_ref = attn_fwd_ref(to64(x["q"]), to64(x["k"]), to64(x["v"]), w.scale, True)
+    check_o_lse(to64(o), to64(lse), o_ref, lse_ref, "many units causal d128")
+
+
+def test_large_scores_rescaling():
+    # peaked rows with a growing max: exercises the conditional O rescale
+    w = Workload("peaked", 1, 2, 1024, 64, "bf16", True, 0.5, False, seed=9)
+    x = make_inputs(w, with_grad=False)
+    ramp = torch.linspace(0.2, 3.0, 1024).view(1, 1, 1024, 1)
+    x["k"] = (x["k"].float() * ramp).to(torch.bfloat16)
+    x, o, lse = _run(w, x)
+    o_ref, lse_ref = attn_fwd_ref(to64(x["q"]), to64(x["k"]), to64(x["v"]), w.scale, True)
+    check_o_lse(to64(o), to64(lse), o_ref, lse_ref, "peaked")
+
+
+def test_tiny_fwd_workload_full():
+    w = workload("tiny_fwd")
+    x, o, lse = _run(w)
+    o_ref, lse_ref = attn_fwd_ref(to64(x["q"]), to64(x["k"]), to64(x["v"]), w.scale, w.causal)
+    check_o_lse(to64(o), to64(lse), o_ref, lse_ref, "tiny_fwd")
+
+
+def test_gpt2_batch_forward_full():
+    w = workload("gpt2_batch")
+    x, o, lse = _run(w)
+    o_ref, lse_ref = attn_fwd_ref(to64(x["q"]), to64(x["k"]), to64(x["v"]), w.scale, w.causal)
+    check_o_lse(to64(o), to64(lse), o_ref, lse_ref, "gpt2_batch")
+
+
+def _sampled_check(name, heads=None, n_random=512):
+    w = workload(name)
+    x, o, lse = _run(w)
+    rng = np.random.default_rng(0)
+    q, k, v = x["q"], x["k"], x["v"]
+    o64, lse64 = o.cpu(), lse.cpu()
+    pairs = [(b, h) for b in range(w.B) for h in range(w.H)]
+    if heads is not None:
+        pairs = [pairs[i] for i in sorted(set(int(i) for i in np.linspace(0, len(pairs) - 1, heads)))]
+    errs = []
+    for b, h in pairs:
+        rows = sample_rows(w.N, rng, n_random)
+        o_ref, lse_ref = attn_fwd_rows_ref(to64(q[b, h]), to64(k[b, h]), to64(v[b, h]), w.scale,
+                                           w.causal, rows=rows)
+        errs.append(check_o_lse(to64(o64[b, h, rows]), to64(lse64[b, h, rows]), o_ref, lse_ref,
+                                f"{name} b={b} h={h}"))
+    # every output is finite on the GPU side, sampled or not
+    assert torch.isfinite(o64.float()).all() and torch.isfinite(lse64).all()
+    return errs
+
+
+def test_seq4k_fp16_sampled():
+    _sampled_check("seq4k_fp16")
+
+
+def test_trading_day_sampled():
+    _sampled_check("trading_day")
+
+
+@pytest.mark.parametrize("name", ["d128_n2048_nc", "d128_n2048_causal", "d128_n8192_nc",
+                                  "d128_n8192_causal", "d128_n16384_nc", "d128_n16384_causal"])
+def test_d128_sweep_sampled(name):
+    _sampled_check(name, heads=4, n_random=256)
+
+
+def test_constant_value_at_full_size():
+    # no oracle needed: V constant per channel => O equals that constant
+    w = workload("d128_n8192_causal")
+    x = make_inputs(w, with_grad=False)
+    c = torch.randn(w.d, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16)
+    x["v"] = c.view(1, 1, 1, -1).expand_as(x["v"]).contiguous()
+    _, o, lse = _run(w, x)
+    err = (o.float() - c.float().cuda()).abs().max().item()
+    assert err <= 1e-2, err
