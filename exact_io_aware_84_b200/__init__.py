@@ -26,6 +26,7 @@ __all__ = [
     "fa_last_device_status",
     "fa_debug_set_wait_limit_ms",
     "fa_debug_set_flags",
+    "fa_debug_exp2_poly",
     "fa_version",
     "FA_OK",
     "FA_ERR_INVALID_ARG",
@@ -62,6 +63,7 @@ _SIGNATURES = {
     "fa_last_device_status": (_c_int, [_vp]),
     "fa_debug_set_wait_limit_ms": (_c_int, [_c_int]),
     "fa_debug_set_flags": (_c_int, [_c_int]),
+    "fa_debug_exp2_poly": (_c_int, [_vp, _vp, _c_int, _vp]),
     "fa_version": (ctypes.c_char_p, []),
 }
 EXPORTED_SYMBOLS = tuple(_SIGNATURES)
@@ -117,6 +119,18 @@ def fa_debug_set_wait_limit_ms(ms: int) -> int:
 
 def fa_debug_set_flags(flags: int) -> int:
     return load_library().fa_debug_set_flags(int(flags))
+
+
+def fa_debug_exp2_poly(x, stream=None):
+    """2^x by the library's FMA-pipe polynomial (diagnostics); x: CUDA float32."""
+    torch = _torch()
+    if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA float32 tensor")
+    y = torch.empty_like(x)
+    st = load_library().fa_debug_exp2_poly(x.data_ptr(), y.data_ptr(), x.numel(), _stream_handle(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_debug_exp2_poly")
+    return y
 
 
 def _torch():

@@ -320,10 +320,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool key_ok = key < p.N;
       for (int i = bu.i0; i <= bu.i1; ++i, ++q_iter) {
         const uint32_t st = q_iter & 1;
-        if (!mbar_wait(BAR(L::kQFull + st), (q_iter >> 1) & 1, wc)) { ok = false; break; }
+        ok = warp_all(mbar_wait(BAR(L::kQFull + st), (q_iter >> 1) & 1, wc));
+        if (!ok) break;
         const float* lse2 = reinterpret_cast<const float*>(gbase + L::kVecOff + st * L::kVecStage);
         const float* dvec = lse2 + BR;
-        if (!mbar_wait(BAR(L::kSFull), s_cnt & 1, wc)) { ok = false; break; }
+        ok = warp_all(mbar_wait(BAR(L::kSFull), s_cnt & 1, wc));
+        if (!ok) break;
         ++s_cnt;
         tc_fence_after();
         const int q0 = i * BR;
@@ -350,10 +352,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_before();
         mbar_arrive(BAR(L::kPFull));
         // dS^T = P^T o (dP^T - D)
-        if (!mbar_wait(BAR(L::kDPFull), dp_cnt & 1, wc)) { ok = false; break; }
+        ok = warp_all(mbar_wait(BAR(L::kDPFull), dp_cnt & 1, wc));
+        if (!ok) break;
         ++dp_cnt;
         tc_fence_after();
-        if (ds_cnt > 0 && !mbar_wait(BAR(L::kDSEmpty), (ds_cnt - 1) & 1, wc)) { ok = false; break; }
+        ok = warp_all(ds_cnt == 0 || mbar_wait(BAR(L::kDSEmpty), (ds_cnt - 1) & 1, wc));
+        if (!ok) break;
         ++ds_cnt;
         uint32_t dsk[BR / 2];
 #pragma unroll
@@ -411,7 +415,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
       const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
       for (int i = bu.i0; i <= bu.i1; ++i) {
-        if (!mbar_wait(BAR(L::kDQFull), dq_cnt & 1, wc)) { ok = false; break; }
+        ok = warp_all(mbar_wait(BAR(L::kDQFull), dq_cnt & 1, wc));
+        if (!ok) break;
         ++dq_cnt;
         tc_fence_after();
         // 64 fp32 columns per lane: d=64 -> lane = query, cols = dims;
@@ -463,7 +468,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       if (!ok) break;
       // dK, dV of this key tile: lane = key
-      if (!mbar_wait(BAR(L::kAccFull), unit_iter & 1, wc)) { ok = false; break; }
+      ok = warp_all(mbar_wait(BAR(L::kAccFull), unit_iter & 1, wc));
+      if (!ok) break;
       tc_fence_after();
       const int key = bu.jk * kBlockN + t;
       const bool in_range = key < p.N;

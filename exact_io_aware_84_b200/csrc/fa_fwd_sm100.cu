@@ -33,6 +33,13 @@ constexpr int kFwdThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only if max grows > 2^8
+// Which of the 8 element pairs in every 16 columns take exp2 on the FMA pipe
+// (exp2_poly) instead of the MUFU unit: bit k set = pair k.  Balances the
+// two pipes; the MUFU alone caps the softmax at 16 exponentials/clock/SM.
+#ifndef FA_FWD_POLY_PAIR_MASK
+#define FA_FWD_POLY_PAIR_MASK 0x00
+#endif
+constexpr uint32_t kPolyPairMask = FA_FWD_POLY_PAIR_MASK;
 // Register split.  Launch: 384 threads x 168 registers.  Warp w runs on SM
 // sub-partition w % 4, which therefore holds warps {k, k+4, k+8}: two softmax
 // warps and one warp of the producer/MMA warpgroup.  Each sub-partition's
@@ -289,7 +296,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const int row = ui.r0(t) + r_in;
       float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; j < nb; ++j) {
-        if (!mbar_wait(BAR(L::kSFull + t), s_cnt & 1, wc)) { ok = false; break; }
+        ok = warp_all(mbar_wait(BAR(L::kSFull + t), s_cnt & 1, wc));
+        if (!ok) break;
         ++s_cnt;
         tc_fence_after();
         uint32_t sr[kBlockN];
@@ -309,43 +317,60 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int c = 0; c < kBlockN; ++c)
             if (kbase + c >= p.N) s[c] = -INFINITY;
         }
-        float mx = s[0];
+        // row max: eight independent partial maxima, three inputs per step
+        float pm[8];
 #pragma unroll
-        for (int c = 1; c < kBlockN; ++c) mx = fmaxf(mx, s[c]);
+        for (int a = 0; a < 8; ++a) pm[a] = fmaxf(s[a], s[a + 8]);
+#pragma unroll
+        for (int c = 16; c + 16 <= kBlockN; c += 16)
+#pragma unroll
+          for (int a = 0; a < 8; ++a) pm[a] = fmax3(pm[a], s[c + a], s[c + a + 8]);
+        const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
         const float m_new = fmaxf(m_run, mx * sl2);
         if (j == 0) {
           m_run = (m_new == -INFINITY) ? 0.f : m_new;
-        } else if (m_new > m_run + kRescaleThreshold) {
-          const float alpha = ex2_approx(m_run - m_new);
-          l_run *= alpha;
-          m_run = m_new;
-          // O_t was last written by PV of tile j-1, which completed before
-          // S_j was signalled (tcgen05 ops of one thread complete in order).
+        } else {
+          // The rescale touches tensor memory with warp-collective
+          // instructions, so the whole warp takes the branch when any of its
+          // rows needs it; rows that do not keep their max and use alpha = 1.
+          const bool need = m_new > m_run + kRescaleThreshold;
+          if (__any_sync(0xffffffffu, need)) {
+            const float alpha = need ? ex2_approx(m_run - m_new) : 1.f;
+            if (need) {
+              l_run *= alpha;
+              m_run = m_new;
+            }
+            // O_t was last written by PV of tile j-1, which completed before
+            // S_j was signalled (tcgen05 ops of one thread complete in order).
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32u * c, o);
-            tmem_wait_ld();
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tO + 32u * c, o);
+              tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tO + 32u * c, o);
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(tO + 32u * c, o);
+            }
           }
         }
         const float neg_m = -m_run;
-        float sum = 0.f;
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int q = 0; q < kBlockN / 32; ++q) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2_approx(fmaf(s[32 * q + 2 * e], sl2, neg_m));
-            const float p1 = ex2_approx(fmaf(s[32 * q + 2 * e + 1], sl2, neg_m));
-            sum += p0 + p1;
+            const float x0 = fmaf(s[32 * q + 2 * e], sl2, neg_m);
+            const float x1 = fmaf(s[32 * q + 2 * e + 1], sl2, neg_m);
+            const bool poly = (kPolyPairMask >> (e & 7)) & 1u;
+            const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
+            const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+            ps[e & 3] += p0 + p1;
             pk[e] = pack2<BF16>(p0, p1);
           }
           tmem_st16(tS + 16u * q, pk);
         }
-        l_run += sum;
+        l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         tmem_wait_st();
         tc_fence_before();
         const bool withhold = (p.debug_flags & 1) && unit_iter == 0 && j == 0 && t == 0;
@@ -353,7 +378,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (!ok) break;
       // ---- epilogue: O / l -> dtype -> global; LSE = (m + log2 l) ln 2
-      if (!mbar_wait(BAR(L::kOFull + t), o_cnt & 1, wc)) { ok = false; break; }
+      ok = warp_all(mbar_wait(BAR(L::kOFull + t), o_cnt & 1, wc));
+      if (!ok) break;
       ++o_cnt;
       tc_fence_after();
       const float inv_l = 1.f / l_run;

@@ -91,6 +91,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   }
 }
 
+// Threads that go on to warp-collective (.sync.aligned) tcgen05 instructions
+// must agree on whether a wait succeeded; a lane that gave up at the deadline
+// while its neighbours saw the phase complete would otherwise diverge there.
+__device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
+
 // Same wait, used while draining after an abort: it ignores the abort flag
 // (the point is to let in-flight copies / MMAs land) but keeps the time limit.
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
@@ -263,6 +268,33 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Base-2 exponential on the FMA pipe, for inputs x <= 64 (the softmax only
+// passes x <= ~8).  Cody-Waite split x = j + f with j = rint(x) (the
+// 1.5 * 2^23 rounding constant) and f in [-0.5, 0.5]; 2^f by a degree-3
+// polynomial fitted for minimax relative error on [-0.5, 0.5] (max relative
+// error 7.5e-5, below the 2^-9 spacing of bf16); 2^j is added into the
+// exponent field.  Inputs below -126 (including -inf) are clamped to -126, so
+// they return ~1e-38 instead of 0.  Used for a fraction of the softmax
+// exponentials to take load off the MUFU unit.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.f);
+  const float kRound = 12582912.f;  // 1.5 * 2^23
+  const float t = x + kRound;       // j in the low mantissa bits (round to nearest)
+  const float j = t - kRound;
+  const float f = x - j;
+  float p = fmaf(0.055171579f, f, 0.24261102f);
+  p = fmaf(p, f, 0.69326097f);
+  p = fmaf(p, f, 0.99992806f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 // Pack two fp32 into one 32-bit word of 16-bit floats: `lo` in bits 0-15.

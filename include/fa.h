@@ -128,6 +128,17 @@ int fa_last_device_status(void* stream);
 int fa_debug_set_wait_limit_ms(int ms);
 int fa_debug_set_flags(int flags);
 
+/*
+ * Diagnostics: y[i] = 2^x[i] computed by the FMA-pipe polynomial the forward
+ * kernel can use for part of its softmax exponentials (Cody-Waite split into
+ * integer and fractional part, degree-3 minimax polynomial for 2^f on
+ * [-0.5, 0.5], relative error < 1e-4 for -126 <= x <= 64; inputs below -126
+ * give about 1e-38).  x, y: device float arrays of n elements.  One launch on
+ * `stream`.  Not part of the attention computation's interface; it exists so
+ * that the polynomial can be checked against the hardware exponential.
+ */
+int fa_debug_exp2_poly(const float* x, float* y, int n, void* stream);
+
 /* Version string of the library build. */
 const char* fa_version(void);
 
