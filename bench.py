@@ -33,6 +33,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 DEFAULT_WORKLOAD = "gpt2_batch"  # B=8 H=12 N=1024 d=64 bf16 causal, forward + backward
+TARGET_WORKLOAD = "d128_n8192_nc"  # B=2 H=16 N=8192 d=128 bf16 non-causal
 METRIC = "attention fwd/bwd TFLOP/s on 1 B200 (bf16); % of dense BF16 tensor peak"
 L2_FLUSH_BYTES = 256 << 20
 
@@ -46,6 +47,7 @@ def _args():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-target", action="store_true")
     return ap.parse_args()
 
 
@@ -320,6 +322,8 @@ def run_native(args):
                         "measured_sustained": value / world / peaks["bf16_tflops_sustained"],
                         "datasheet_2250": value / world / 2250.0},
     }
+    if not args.no_target and w.name != TARGET_WORKLOAD:
+        line["north_star_target"] = _target_fwd(fa, torch, dev, stream, flush, peaks, args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, heads, el = _oracle_sample(w, 12.0)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": _cpu_threads(), "kind": "oracle",
@@ -331,6 +335,33 @@ def run_native(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def _target_fwd(fa, torch, dev, stream, flush, peaks, args):
+    """Forward-only TFLOP/s on the d=128, N=8192, non-causal workload (the
+    throughput target: >= 60% of dense BF16 peak), timed like the main leg."""
+    from exact_io_aware_84_b200.inputs import make_inputs, workload
+    from exact_io_aware_84_b200.metrics import attn_fwd_flops
+    w = workload(TARGET_WORKLOAD)
+    x = make_inputs(w, with_grad=False)
+    g = {k: v.to(dev) for k, v in x.items()}
+    o = torch.empty_like(g["q"])
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    for _ in range(max(3, args.warmup)):
+        fa.fa_fwd(g["q"], g["k"], g["v"], o, lse, scale=w.scale, causal=w.causal, stream=stream)
+    ms = []
+    for _ in range(max(5, args.steps)):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        fa.fa_fwd(g["q"], g["k"], g["v"], o, lse, scale=w.scale, causal=w.causal, stream=stream)
+        e.record(stream)
+        ms.append((s, e))
+    torch.cuda.synchronize()
+    t = statistics.mean(a.elapsed_time(b) for a, b in ms)
+    tf = attn_fwd_flops(w.B, w.H, w.N, w.d, w.causal) / (t * 1e-3) / 1e12
+    return {"workload": w.name, "fwd_ms": t, "fwd_tflops": tf, "frac_of_measured_burst": tf / peaks["bf16_tflops"],
+            "target_frac": 0.60}
 
 
 def _e2e(fa, torch, w, x, dev, stream, flops, world, args):

@@ -50,6 +50,8 @@ FA_ERR_NO_DEVICE = 7
 
 FA_BF16 = 0
 FA_FP16 = 1
+FA_BF16_O_F32 = 2  # 16-bit q, k, v, dO and gradients; O stored in float32
+FA_FP16_O_F32 = 3
 
 _c_int, _c_float, _vp, _sz = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
@@ -149,31 +151,38 @@ def fa_last_device_status(stream=None) -> int:
     return load_library().fa_last_device_status(_stream_handle(stream))
 
 
-def _dtype_code(t) -> int:
+def _dtype_code(t, o=None) -> int:
+    """Storage code for 16-bit tensor ``t``; O in float32 selects the *_O_F32 codes."""
     torch = _torch()
+    o32 = o is not None and o.dtype == torch.float32
     if t.dtype == torch.bfloat16:
-        return FA_BF16
+        return FA_BF16_O_F32 if o32 else FA_BF16
     if t.dtype == torch.float16:
-        return FA_FP16
+        return FA_FP16_O_F32 if o32 else FA_FP16
     raise TypeError(f"unsupported dtype {t.dtype}: expected bfloat16 or float16")
 
 
-def _check_bhnd(name, t, ref=None):
+def _check_bhnd(name, t, ref=None, allow_f32=False):
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if t.dim() != 4:
         raise ValueError(f"{name} must be [B, H, N, d], got shape {tuple(t.shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
-    if ref is not None and (t.shape != ref.shape or t.dtype != ref.dtype or t.device != ref.device):
-        raise ValueError(f"{name} must match q in shape, dtype and device")
+    if ref is not None:
+        same_type = t.dtype == ref.dtype or (allow_f32 and t.dtype == _torch().float32)
+        if t.shape != ref.shape or not same_type or t.device != ref.device:
+            raise ValueError(f"{name} must match q in shape, dtype and device")
 
 
-def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: bool = False, stream=None):
+def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: bool = False, stream=None,
+           o_fp32: bool = False):
     """O = softmax(scale Q K^T [causal]) V and LSE (float32, natural log).
 
     q, k, v: [B, H, N, d] contiguous CUDA tensors (bf16 or fp16).  ``o`` and
-    ``lse`` may be preallocated ([B,H,N,d] same dtype; [B,H,N] float32).
+    ``lse`` may be preallocated ([B,H,N,d]; [B,H,N] float32).  O has q's
+    dtype unless ``o`` is a float32 tensor or ``o_fp32`` is set, in which case
+    it is stored in float32 (see the storage codes in include/fa.h).
     """
     torch = _torch()
     _check_bhnd("q", q)
@@ -183,15 +192,15 @@ def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: boo
     if scale is None:
         scale = 1.0 / float(d) ** 0.5
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty(q.shape, dtype=torch.float32 if o_fp32 else q.dtype, device=q.device)
     else:
-        _check_bhnd("o", o, q)
+        _check_bhnd("o", o, q, allow_f32=True)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     elif lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous float32 [B, H, N] tensor")
     st = load_library().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                               B, H, N, d, float(scale), int(bool(causal)), _dtype_code(q),
+                               B, H, N, d, float(scale), int(bool(causal)), _dtype_code(q, o),
                                _stream_handle(stream))
     if st != FA_OK:
         raise FAError(st, "fa_fwd")
@@ -207,7 +216,7 @@ def fa_bwd(q, k, v, o, do, lse, dq=None, dk=None, dv=None, workspace=None,
     """dQ, dK, dV of L with dL/dO = ``do``, recomputing P from Q, K and LSE."""
     torch = _torch()
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
-        _check_bhnd(name, t, None if name == "q" else q)
+        _check_bhnd(name, t, None if name == "q" else q, allow_f32=(name == "o"))
     B, H, N, d = q.shape
     if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous float32 [B, H, N] tensor")
@@ -224,7 +233,7 @@ def fa_bwd(q, k, v, o, do, lse, dq=None, dk=None, dv=None, workspace=None,
     st = load_library().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
                                lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                                workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                               B, H, N, d, float(scale), int(bool(causal)), _dtype_code(q),
+                               B, H, N, d, float(scale), int(bool(causal)), _dtype_code(q, o),
                                _stream_handle(stream))
     if st != FA_OK:
         raise FAError(st, "fa_bwd")

@@ -87,7 +87,8 @@ int check_common(int B, int H, int N, int d, float scale, int dtype) {
   if (B <= 0 || H <= 0 || N <= 0) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || scale > 3.0e38f) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_UNSUPPORTED;
+  if (dtype != FA_BF16 && dtype != FA_FP16 && dtype != FA_BF16_O_F32 && dtype != FA_FP16_O_F32)
+    return FA_ERR_UNSUPPORTED;
   const long long total = (long long)B * H * ((long long)N + 255) * d;
   if (total >= (1ll << 31)) return FA_ERR_INVALID_ARG;
   return FA_OK;
@@ -163,7 +164,8 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
     return FA_ERR_MISALIGNED;
   DeviceInfo di;
   if ((st = device_info(&di)) != FA_OK) return st;
-  const bool bf16 = dtype == FA_BF16;
+  const bool bf16 = dtype == FA_BF16 || dtype == FA_BF16_O_F32;
+  const bool o32 = dtype == FA_BF16_O_F32 || dtype == FA_FP16_O_F32;
   const int bh = B * H;
   CUtensorMap tq, tk, tv;
   if (encode_tile_map(&tq, q, bh, N, d, bf16, kBlockM) != FA_OK ||
@@ -183,7 +185,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.debug_flags = g_debug_flags.load();
   if (!(p.status = status_ptr())) return FA_ERR_CUDA;
   const int grid = p.n_units < di.sms ? p.n_units : di.sms;
-  cudaError_t e = launch_fwd(d, bf16, causal != 0, tq, tk, tv, p, grid, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_fwd(d, bf16, o32, causal != 0, tq, tk, tv, p, grid, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -209,7 +211,8 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_MISALIGNED;
   DeviceInfo di;
   if ((st = device_info(&di)) != FA_OK) return st;
-  const bool bf16 = dtype == FA_BF16;
+  const bool bf16 = dtype == FA_BF16 || dtype == FA_BF16_O_F32;
+  const bool o32 = dtype == FA_BF16_O_F32 || dtype == FA_FP16_O_F32;
   const int bh = B * H;
   BwdParams p{};
   p.o = o;
@@ -240,7 +243,7 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
       encode_tile_map(&tdo, dout, bh, N, d, bf16, q_rows) != FA_OK)
     return FA_ERR_CUDA;
   const int grid = p.n_units < di.sms ? p.n_units : di.sms;
-  cudaError_t e = launch_bwd(d, bf16, causal != 0, tq, tk, tv, tdo, p, grid, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_bwd(d, bf16, o32, causal != 0, tq, tk, tv, tdo, p, grid, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

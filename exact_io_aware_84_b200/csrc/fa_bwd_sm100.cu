@@ -511,8 +511,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // D_i = sum_c dO_ic O_ic; lse2_i = LSE_i * log2(e); both +0 / +inf on the
-// padding rows N..n_pad-1; dQacc rows zeroed.  One warp per row.
-template <int D, bool BF16>
+// padding rows N..n_pad-1; dQacc rows zeroed.  One warp per row.  O is read
+// as 16-bit, or as fp32 for the O32 storage codes.
+template <int D, bool BF16, bool O32>
 __global__ void __launch_bounds__(256) fa_bwd_prep(const BwdParams p) {
   const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -520,37 +521,45 @@ __global__ void __launch_bounds__(256) fa_bwd_prep(const BwdParams p) {
   if (warp_global >= total) return;
   const int bh = warp_global / p.n_pad;
   const int row = warp_global % p.n_pad;
+  constexpr int PER = D / 32;  // elements per lane (2 or 4)
   float acc = 0.f;
   if (row < p.N) {
-    const size_t off = ((size_t)bh * p.N + row) * D;
-    constexpr int PER = D / 32;  // elements per lane (2 or 4)
-    const uint8_t* o8 = reinterpret_cast<const uint8_t*>(p.o) + off * 2 + lane * PER * 2;
-    const uint8_t* d8 = reinterpret_cast<const uint8_t*>(p.dout) + off * 2 + lane * PER * 2;
-    uint32_t ow[PER / 2], dw[PER / 2];
+    const size_t off = ((size_t)bh * p.N + row) * D + (size_t)lane * PER;
+    const uint32_t* d32 = reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(p.dout) + off * 2);
+    float ov[PER], dv[PER];
 #pragma unroll
     for (int e = 0; e < PER / 2; ++e) {
-      ow[e] = reinterpret_cast<const uint32_t*>(o8)[e];
-      dw[e] = reinterpret_cast<const uint32_t*>(d8)[e];
-    }
-#pragma unroll
-    for (int e = 0; e < PER / 2; ++e) {
-      float a0, a1, b0, b1;
+      const uint32_t w = d32[e];
       if constexpr (BF16) {
-        a0 = __uint_as_float(ow[e] << 16);
-        a1 = __uint_as_float(ow[e] & 0xFFFF0000u);
-        b0 = __uint_as_float(dw[e] << 16);
-        b1 = __uint_as_float(dw[e] & 0xFFFF0000u);
+        dv[2 * e] = __uint_as_float(w << 16);
+        dv[2 * e + 1] = __uint_as_float(w & 0xFFFF0000u);
       } else {
-        const __half2 ha = *reinterpret_cast<const __half2*>(&ow[e]);
-        const __half2 hb = *reinterpret_cast<const __half2*>(&dw[e]);
-        a0 = __low2float(ha);
-        a1 = __high2float(ha);
-        b0 = __low2float(hb);
-        b1 = __high2float(hb);
+        const __half2 h = *reinterpret_cast<const __half2*>(&w);
+        dv[2 * e] = __low2float(h);
+        dv[2 * e + 1] = __high2float(h);
       }
-      acc = fmaf(a0, b0, acc);
-      acc = fmaf(a1, b1, acc);
     }
+    if constexpr (O32) {
+      const float* o32p = reinterpret_cast<const float*>(p.o) + off;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) ov[e] = o32p[e];
+    } else {
+      const uint32_t* o16 = reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(p.o) + off * 2);
+#pragma unroll
+      for (int e = 0; e < PER / 2; ++e) {
+        const uint32_t w = o16[e];
+        if constexpr (BF16) {
+          ov[2 * e] = __uint_as_float(w << 16);
+          ov[2 * e + 1] = __uint_as_float(w & 0xFFFF0000u);
+        } else {
+          const __half2 h = *reinterpret_cast<const __half2*>(&w);
+          ov[2 * e] = __low2float(h);
+          ov[2 * e + 1] = __high2float(h);
+        }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc = fmaf(ov[e], dv[e], acc);
   }
 #pragma unroll
   for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
@@ -580,12 +589,15 @@ __global__ void __launch_bounds__(256) fa_bwd_dq(const BwdParams p) {
 }
 
 template <int D, bool BF16, bool CAUSAL>
-cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+cudaError_t launch_bwd_t(bool o32, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& tdo, const BwdParams& p, int grid, cudaStream_t st) {
   {
     const long long warps = (long long)p.bh * p.n_pad;
     const int blocks = (int)((warps * 32 + 255) / 256);
-    fa_bwd_prep<D, BF16><<<blocks, 256, 0, st>>>(p);
+    if (o32)
+      fa_bwd_prep<D, BF16, true><<<blocks, 256, 0, st>>>(p);
+    else
+      fa_bwd_prep<D, BF16, false><<<blocks, 256, 0, st>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -610,11 +622,11 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 int bwd_threads() { return kBwdThreads; }
 
-cudaError_t launch_bwd(int d, bool bf16, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
+cudaError_t launch_bwd(int d, bool bf16, bool o32, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p, int grid,
                        cudaStream_t st) {
 #define FA_BWD_CASE(DD, BB, CC) \
-  if (d == DD && bf16 == BB && causal == CC) return launch_bwd_t<DD, BB, CC>(tq, tk, tv, tdo, p, grid, st);
+  if (d == DD && bf16 == BB && causal == CC) return launch_bwd_t<DD, BB, CC>(o32, tq, tk, tv, tdo, p, grid, st);
   FA_BWD_CASE(64, true, false)
   FA_BWD_CASE(64, true, true)
   FA_BWD_CASE(64, false, false)

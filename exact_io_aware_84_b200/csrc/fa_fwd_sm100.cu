@@ -45,8 +45,8 @@ constexpr uint32_t kPolyPairMask = FA_FWD_POLY_PAIR_MASK;
 // warps and one warp of the producer/MMA warpgroup.  Each sub-partition's
 // share after the split must not exceed its launch share (3 x 168).
 constexpr int kLaunchRegs = 168;
-constexpr int kRegsSoftmax = 224;
-constexpr int kRegsOther = 56;
+constexpr int kRegsSoftmax = 216;
+constexpr int kRegsOther = 72;
 static_assert(2 * kRegsSoftmax + kRegsOther <= 3 * kLaunchRegs, "register split exceeds a sub-partition's pool");
 
 template <int D>
@@ -118,7 +118,7 @@ __device__ __forceinline__ uint64_t v_desc(uint32_t tile, int kstep) {
   return make_sdesc_sw128(tile + (uint32_t)kstep * 2048, kBlockN * 128, 1024);
 }
 
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool O32, bool CAUSAL>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -301,40 +301,75 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         ++s_cnt;
         tc_fence_after();
         uint32_t sr[kBlockN];
-#pragma unroll
-        for (int c = 0; c < kBlockN / 32; ++c) tmem_ld32(tS + 32u * c, sr + 32 * c);
-        tmem_wait_ld();
-        float s[kBlockN];
-#pragma unroll
-        for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(sr[c]);
         const int kbase = j * kBlockN;
-        if (CAUSAL && j == nb - 1) {
-#pragma unroll
-          for (int c = 0; c < kBlockN; ++c)
-            if (kbase + c > row) s[c] = -INFINITY;
-        } else if (!CAUSAL && kbase + kBlockN > p.N) {
-#pragma unroll
-          for (int c = 0; c < kBlockN; ++c)
-            if (kbase + c >= p.N) s[c] = -INFINITY;
-        }
-        // row max: eight independent partial maxima, three inputs per step
+        // columns of this tile that must be masked: keys in the future of a
+        // row (causal diagonal tile) or past the sequence end (ragged tail)
+        const bool diag = CAUSAL && j == nb - 1;
+        const bool tail = !CAUSAL && kbase + kBlockN > p.N;
+        const int limit = diag ? (row - kbase) : (p.N - 1 - kbase);  // last valid column
+        auto masked = [&](int c) -> float {
+          const float v = __uint_as_float(sr[c]);
+          return ((diag || tail) && c > limit) ? -INFINITY : v;
+        };
         float pm[8];
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};
+        // exp2(S*scale*log2e - m) for one 32-column chunk; P -> tensor memory
+        auto exp_chunk = [&](int q, float neg_m) {
 #pragma unroll
-        for (int a = 0; a < 8; ++a) pm[a] = fmaxf(s[a], s[a + 8]);
+          for (int h = 0; h < 2; ++h) {
+            uint32_t pk[8];
 #pragma unroll
-        for (int c = 16; c + 16 <= kBlockN; c += 16)
+            for (int e = 0; e < 8; ++e) {
+              const int c = 32 * q + 16 * h + 2 * e;
+              const float x0 = fmaf(masked(c), sl2, neg_m);
+              const float x1 = fmaf(masked(c + 1), sl2, neg_m);
+              const bool poly = (kPolyPairMask >> e) & 1u;
+              const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
+              const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+              ps[e & 3] += p0 + p1;
+              pk[e] = pack2<BF16>(p0, p1);
+            }
+            tmem_st8(tS + 16u * q + 8u * h, pk);
+          }
+        };
+        auto chunk_max = [&](int q) {
 #pragma unroll
-          for (int a = 0; a < 8; ++a) pm[a] = fmax3(pm[a], s[c + a], s[c + a + 8]);
-        const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
-        const float m_new = fmaxf(m_run, mx * sl2);
+          for (int a = 0; a < 8; ++a) {
+            const float m3 = fmax3(masked(32 * q + a), masked(32 * q + a + 8), masked(32 * q + a + 16));
+            pm[a] = (q == 0) ? fmaxf(m3, masked(32 * q + a + 24)) : fmax3(pm[a], m3, masked(32 * q + a + 24));
+          }
+        };
         if (j == 0) {
-          m_run = (m_new == -INFINITY) ? 0.f : m_new;
+          // first tile: the running max must come first
+#pragma unroll
+          for (int c = 0; c < kBlockN / 32; ++c) tmem_ld32(tS + 32u * c, sr + 32 * c);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < kBlockN / 32; ++q) chunk_max(q);
+          const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+          m_run = (mx == -INFINITY) ? 0.f : mx * sl2;
+#pragma unroll
+          for (int q = 0; q < kBlockN / 32; ++q) exp_chunk(q, -m_run);
         } else {
-          // The rescale touches tensor memory with warp-collective
-          // instructions, so the whole warp takes the branch when any of its
-          // rows needs it; rows that do not keep their max and use alpha = 1.
+          // Later tiles: exponentiate against the running max while the next
+          // 32-column chunk is still being read from tensor memory; check the
+          // new row max afterwards.
+          tmem_ld32(tS, sr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < kBlockN / 32; ++q) {
+            if (q + 1 < kBlockN / 32) tmem_ld32(tS + 32u * (q + 1), sr + 32 * (q + 1));
+            chunk_max(q);
+            exp_chunk(q, -m_run);
+            if (q + 1 < kBlockN / 32) tmem_wait_ld();
+          }
+          const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+          const float m_new = mx * sl2;
           const bool need = m_new > m_run + kRescaleThreshold;
           if (__any_sync(0xffffffffu, need)) {
+            // Rare: a row's max grew by more than 2^8.  The whole warp takes
+            // this branch (tensor-memory access is warp-collective); rows that
+            // do not need it keep their max and use alpha = 1.
             const float alpha = need ? ex2_approx(m_run - m_new) : 1.f;
             if (need) {
               l_run *= alpha;
@@ -351,24 +386,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
               tmem_st32(tO + 32u * c, o);
             }
-          }
-        }
-        const float neg_m = -m_run;
-        float ps[4] = {0.f, 0.f, 0.f, 0.f};
+            // redo P (and its row sum) against the updated max
+            tmem_wait_st();
 #pragma unroll
-        for (int q = 0; q < kBlockN / 32; ++q) {
-          uint32_t pk[16];
+            for (int a = 0; a < 4; ++a) ps[a] = 0.f;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float x0 = fmaf(s[32 * q + 2 * e], sl2, neg_m);
-            const float x1 = fmaf(s[32 * q + 2 * e + 1], sl2, neg_m);
-            const bool poly = (kPolyPairMask >> (e & 7)) & 1u;
-            const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
-            const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
-            ps[e & 3] += p0 + p1;
-            pk[e] = pack2<BF16>(p0, p1);
+            for (int q = 0; q < kBlockN / 32; ++q) exp_chunk(q, -m_run);
           }
-          tmem_st16(tS + 16u * q, pk);
         }
         l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         tmem_wait_st();
@@ -384,20 +408,33 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       const bool in_range = row < p.N;
-      uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + ((size_t)ui.bh * p.N + (size_t)(in_range ? row : 0)) * D * 2;
+      constexpr int kOBytes = O32 ? 4 : 2;
+      uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + ((size_t)ui.bh * p.N + (size_t)(in_range ? row : 0)) * D * kOBytes;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         tmem_ld32(tO + 32u * c, o);
         tmem_wait_ld();
-        uint32_t w[16];
+        if constexpr (O32) {
+          if (in_range) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 128);
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = pack2<BF16>(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-        if (in_range) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_uint4(__float_as_uint(__uint_as_float(o[4 * e]) * inv_l),
+                                  __float_as_uint(__uint_as_float(o[4 * e + 1]) * inv_l),
+                                  __float_as_uint(__uint_as_float(o[4 * e + 2]) * inv_l),
+                                  __float_as_uint(__uint_as_float(o[4 * e + 3]) * inv_l));
+          }
+        } else {
+          uint32_t w[16];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack2<BF16>(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+          if (in_range) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          }
         }
       }
       tc_fence_before();
@@ -415,10 +452,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 }
 
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool O32, bool CAUSAL>
 cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const FwdParams& p, int grid, cudaStream_t st) {
-  auto kern = fa_fwd_kernel<D, BF16, CAUSAL>;
+  auto kern = fa_fwd_kernel<D, BF16, O32, CAUSAL>;
   constexpr int smem = FwdLayout<D>::kAlloc;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -426,23 +463,30 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   return cudaGetLastError();
 }
 
+template <int D, bool BF16, bool O32>
+cudaError_t launch_fwd_c(bool causal, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const FwdParams& p, int grid, cudaStream_t st) {
+  return causal ? launch_fwd_t<D, BF16, O32, true>(tq, tk, tv, p, grid, st)
+                : launch_fwd_t<D, BF16, O32, false>(tq, tk, tv, p, grid, st);
+}
+
+template <int D>
+cudaError_t launch_fwd_d(bool bf16, bool o32, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
+                         const CUtensorMap& tv, const FwdParams& p, int grid, cudaStream_t st) {
+  if (bf16) return o32 ? launch_fwd_c<D, true, true>(causal, tq, tk, tv, p, grid, st)
+                       : launch_fwd_c<D, true, false>(causal, tq, tk, tv, p, grid, st);
+  return o32 ? launch_fwd_c<D, false, true>(causal, tq, tk, tv, p, grid, st)
+             : launch_fwd_c<D, false, false>(causal, tq, tk, tv, p, grid, st);
+}
+
 }  // namespace
 
 int fwd_threads() { return kFwdThreads; }
 
-cudaError_t launch_fwd(int d, bool bf16, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
+cudaError_t launch_fwd(int d, bool bf16, bool o32, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const FwdParams& p, int grid, cudaStream_t st) {
-#define FA_FWD_CASE(DD, BB, CC) \
-  if (d == DD && bf16 == BB && causal == CC) return launch_fwd_t<DD, BB, CC>(tq, tk, tv, p, grid, st);
-  FA_FWD_CASE(64, true, false)
-  FA_FWD_CASE(64, true, true)
-  FA_FWD_CASE(64, false, false)
-  FA_FWD_CASE(64, false, true)
-  FA_FWD_CASE(128, true, false)
-  FA_FWD_CASE(128, true, true)
-  FA_FWD_CASE(128, false, false)
-  FA_FWD_CASE(128, false, true)
-#undef FA_FWD_CASE
+  if (d == 64) return launch_fwd_d<64>(bf16, o32, causal, tq, tk, tv, p, grid, st);
+  if (d == 128) return launch_fwd_d<128>(bf16, o32, causal, tq, tk, tv, p, grid, st);
   return cudaErrorInvalidValue;
 }
 

@@ -12,7 +12,7 @@ constexpr int kBlockM = 128;  // query rows per Q tile (tcgen05 M)
 constexpr int kBlockN = 128;  // keys per K/V tile
 
 struct FwdParams {
-  void* o;             // [B*H, N, D] dtype
+  void* o;             // [B*H, N, D] 16-bit, or fp32 when the O32 variant runs
   float* lse;          // [B*H, N] fp32
   int N;               // sequence length
   int bh;              // B*H
@@ -26,7 +26,7 @@ struct FwdParams {
 };
 
 struct BwdParams {
-  const void* o;       // forward output, [B*H, N, D]
+  const void* o;       // forward output, [B*H, N, D] (16-bit, or fp32 for O32)
   const void* dout;    // dO, [B*H, N, D]
   const float* lse;    // [B*H, N]
   void* dq;            // [B*H, N, D]
@@ -47,10 +47,10 @@ struct BwdParams {
 };
 
 // Launchers (return cudaError_t of the launch).
-cudaError_t launch_fwd(int d, bool bf16, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
+cudaError_t launch_fwd(int d, bool bf16, bool o32, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const FwdParams& p, int grid, cudaStream_t st);
 
-cudaError_t launch_bwd(int d, bool bf16, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
+cudaError_t launch_bwd(int d, bool bf16, bool o32, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p, int grid,
                        cudaStream_t st);
 

@@ -238,6 +238,12 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
@@ -282,11 +288,11 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // 1.5 * 2^23 rounding constant) and f in [-0.5, 0.5]; 2^f by a degree-3
 // polynomial fitted for minimax relative error on [-0.5, 0.5] (max relative
 // error 7.5e-5, below the 2^-9 spacing of bf16); 2^j is added into the
-// exponent field.  Inputs below -126 (including -inf) are clamped to -126, so
-// they return ~1e-38 instead of 0.  Used for a fraction of the softmax
-// exponentials to take load off the MUFU unit.
+// exponent field.  Inputs below -125 (including -inf) are clamped to -125, so
+// every result stays a normal float (they return ~2e-38 instead of 0).  Used
+// for a fraction of the softmax exponentials to take load off the MUFU unit.
 __device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.f);
+  x = fmaxf(x, -125.f);
   const float kRound = 12582912.f;  // 1.5 * 2^23
   const float t = x + kRound;       // j in the low mantissa bits (round to nearest)
   const float j = t - kRound;

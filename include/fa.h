@@ -22,7 +22,9 @@
  * evaluation (delect.ru glossary "FlashAttention", "What is confirmed").
  *
  * Layout.  q, k, v, o, dout, dq, dk, dv: [B, H, N, d] contiguous, row stride d
- * elements, element type `dtype` (FA_BF16 or FA_FP16).  lse: [B, H, N]
+ * elements, element type given by `dtype`: FA_BF16 / FA_FP16 = all of them
+ * bf16 / fp16; FA_BF16_O_F32 / FA_FP16_O_F32 = the same except that o (the
+ * forward's output and the backward's input) is float32.  lse: [B, H, N]
  * contiguous float32, natural log.  Every pointer is a device pointer
  * aligned to 16 bytes.  Supported: d in {64, 128}; N >= 1 (any N: the last
  * tile may be ragged); B >= 1, H >= 1; B*H*N*d < 2^31.
@@ -59,12 +61,21 @@ typedef enum {
   FA_ERR_NO_DEVICE = 7    /* no sm_100 device is current */
 } fa_status;
 
-typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
+/*
+ * Storage types.  With O stored in 16 bits, the backward's row term
+ * D_i = sum_c dO_ic O_ic inherits O's rounding (2^-9 relative for bf16); on
+ * sharply peaked softmax rows dP - D cancels and that rounding reaches dQ at
+ * about 1e-2 relative.  The *_O_F32 codes keep O in float32 (the forward's
+ * own accumulator, normalised) so that D carries only the forward's
+ * arithmetic error; they cost 2 extra bytes per element of O traffic.
+ */
+typedef enum { FA_BF16 = 0, FA_FP16 = 1, FA_BF16_O_F32 = 2, FA_FP16_O_F32 = 3 } fa_dtype;
 
 /*
  * Forward: O = softmax(scale * Q K^T [causal]) V and LSE.
  *   q, k, v : inputs, [B,H,N,d], dtype.
- *   o       : output, [B,H,N,d], dtype (round-to-nearest-even of O).
+ *   o       : output, [B,H,N,d], dtype's O type (16-bit: round-to-nearest-
+ *             even of O; float32 for the *_O_F32 codes).
  *   lse     : output, [B,H,N] float32, LSE_i = ln sum_j exp(S_ij).
  *   scale   : score multiplier (1/sqrt(d) for standard attention).
  *   causal  : non-zero => key j attends to query i only if j <= i
@@ -91,7 +102,8 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  * and the forward's LSE (never storing P):
  *   D_i = sum_c dO_ic O_ic;  dV = P^T dO;  dP = dO V^T;  dS = P o (dP - D);
  *   dQ = scale dS K;  dK = scale dS^T Q.
- *   q, k, v, o, dout : inputs, [B,H,N,d], dtype (o is the forward's output).
+ *   q, k, v, dout    : inputs, [B,H,N,d], dtype.
+ *   o                : input, the forward's output in dtype's O type.
  *   lse              : input, [B,H,N] float32 from fa_fwd.
  *   dq, dk, dv       : outputs, [B,H,N,d], dtype.
  *   workspace        : device buffer of at least fa_bwd_workspace_size()
@@ -132,8 +144,8 @@ int fa_debug_set_flags(int flags);
  * Diagnostics: y[i] = 2^x[i] computed by the FMA-pipe polynomial the forward
  * kernel can use for part of its softmax exponentials (Cody-Waite split into
  * integer and fractional part, degree-3 minimax polynomial for 2^f on
- * [-0.5, 0.5], relative error < 1e-4 for -126 <= x <= 64; inputs below -126
- * give about 1e-38).  x, y: device float arrays of n elements.  One launch on
+ * [-0.5, 0.5], relative error < 1e-4 for -125 <= x <= 64; inputs below -125
+ * are clamped to -125 and give about 2e-38).  x, y: device float arrays of n elements.  One launch on
  * `stream`.  Not part of the attention computation's interface; it exists so
  * that the polynomial can be checked against the hardware exponential.
  */

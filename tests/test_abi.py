@@ -72,6 +72,7 @@ def test_fwd_argument_errors(lib):
     assert _fwd(lib, d=96) == fa.FA_ERR_UNSUPPORTED
     assert _fwd(lib, d=256) == fa.FA_ERR_UNSUPPORTED
     assert _fwd(lib, dtype=7) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd(lib, dtype=4) == fa.FA_ERR_UNSUPPORTED
     assert _fwd(lib, B=1 << 14, H=1 << 10, N=1 << 10) == fa.FA_ERR_INVALID_ARG  # > 2^31 elements
     assert _fwd(lib, k=0x1008) == fa.FA_ERR_MISALIGNED
     assert _fwd(lib, lse=0x1004) == fa.FA_ERR_MISALIGNED

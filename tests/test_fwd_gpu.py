@@ -50,6 +50,23 @@ def test_small_shapes_fp16(N, d, causal):
     check_o_lse(to64(o), to64(lse), o_ref, lse_ref, f"fp16 N={N} d={d} causal={causal}")
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp32_o_output(d, causal):
+    w = Workload("o32", 2, 3, 300, d, "bf16", causal, 1.0 / d ** 0.5, False, seed=17)
+    x = make_inputs(w, with_grad=False)
+    g = {k: v.cuda() for k, v in x.items()}
+    o, lse = fa.fa_fwd(g["q"], g["k"], g["v"], scale=w.scale, causal=causal, o_fp32=True)
+    torch.cuda.synchronize()
+    assert o.dtype == torch.float32 and fa.fa_last_device_status() == fa.FA_OK
+    o_ref, lse_ref = attn_fwd_ref(to64(x["q"]), to64(x["k"]), to64(x["v"]), w.scale, causal)
+    check_o_lse(to64(o), to64(lse), o_ref, lse_ref, "fp32 O")
+    # the same kernel with 16-bit O rounds exactly these values
+    o16, _ = fa.fa_fwd(g["q"], g["k"], g["v"], scale=w.scale, causal=causal)
+    torch.cuda.synchronize()
+    assert torch.equal(o16, o.to(torch.bfloat16))
+
+
 def test_many_units_per_cta():
     # more (head, tile-pair) units than SMs: each persistent CTA runs several
     w = Workload("many", 4, 40, 512, 64, "bf16", False, 0.125, False, seed=3)
@@ -139,10 +156,11 @@ def test_constant_value_at_full_size():
 def test_exp2_polynomial_against_hardware_exp2():
     # the FMA-pipe exponential used for part of the softmax: relative error
     # below 1e-4 (bf16 spacing is 2^-9) over the softmax's input range
-    x = torch.cat([torch.linspace(-126.0, 9.0, 1 << 20), torch.tensor([0.0, -0.5, 0.5, 8.0, -1e-7])]).cuda()
+    x = torch.cat([torch.linspace(-125.0, 9.0, 1 << 20), torch.tensor([0.0, -0.5, 0.5, 8.0, -1e-7])]).cuda()
     y = fa.fa_debug_exp2_poly(x)
     ref = torch.exp2(x.double())
     rel = ((y.double() - ref).abs() / ref).max().item()
     assert rel < 1e-4, rel
-    z = fa.fa_debug_exp2_poly(torch.tensor([-float("inf"), -500.0], device="cuda"))
-    assert (z >= 0).all() and (z < 2e-38).all()
+    # below the clamp (masked scores are -inf) the result is tiny and positive
+    z = fa.fa_debug_exp2_poly(torch.tensor([-float("inf"), -500.0, -125.5], device="cuda"))
+    assert (z > 0).all() and (z < 4e-38).all()
