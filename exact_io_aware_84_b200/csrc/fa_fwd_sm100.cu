@@ -301,75 +301,40 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         ++s_cnt;
         tc_fence_after();
         uint32_t sr[kBlockN];
+#pragma unroll
+        for (int c = 0; c < kBlockN / 32; ++c) tmem_ld32(tS + 32u * c, sr + 32 * c);
+        tmem_wait_ld();
+        float s[kBlockN];
+#pragma unroll
+        for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(sr[c]);
         const int kbase = j * kBlockN;
-        // columns of this tile that must be masked: keys in the future of a
-        // row (causal diagonal tile) or past the sequence end (ragged tail)
-        const bool diag = CAUSAL && j == nb - 1;
-        const bool tail = !CAUSAL && kbase + kBlockN > p.N;
-        const int limit = diag ? (row - kbase) : (p.N - 1 - kbase);  // last valid column
-        auto masked = [&](int c) -> float {
-          const float v = __uint_as_float(sr[c]);
-          return ((diag || tail) && c > limit) ? -INFINITY : v;
-        };
+        if (CAUSAL && j == nb - 1) {
+#pragma unroll
+          for (int c = 0; c < kBlockN; ++c)
+            if (kbase + c > row) s[c] = -INFINITY;
+        } else if (!CAUSAL && kbase + kBlockN > p.N) {
+#pragma unroll
+          for (int c = 0; c < kBlockN; ++c)
+            if (kbase + c >= p.N) s[c] = -INFINITY;
+        }
+        // row max: eight independent partial maxima, three inputs per step
         float pm[8];
-        float ps[4] = {0.f, 0.f, 0.f, 0.f};
-        // exp2(S*scale*log2e - m) for one 32-column chunk; P -> tensor memory
-        auto exp_chunk = [&](int q, float neg_m) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t pk[8];
+        for (int a = 0; a < 8; ++a) pm[a] = fmaxf(s[a], s[a + 8]);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int c = 32 * q + 16 * h + 2 * e;
-              const float x0 = fmaf(masked(c), sl2, neg_m);
-              const float x1 = fmaf(masked(c + 1), sl2, neg_m);
-              const bool poly = (kPolyPairMask >> e) & 1u;
-              const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
-              const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
-              ps[e & 3] += p0 + p1;
-              pk[e] = pack2<BF16>(p0, p1);
-            }
-            tmem_st8(tS + 16u * q + 8u * h, pk);
-          }
-        };
-        auto chunk_max = [&](int q) {
+        for (int c = 16; c + 16 <= kBlockN; c += 16)
 #pragma unroll
-          for (int a = 0; a < 8; ++a) {
-            const float m3 = fmax3(masked(32 * q + a), masked(32 * q + a + 8), masked(32 * q + a + 16));
-            pm[a] = (q == 0) ? fmaxf(m3, masked(32 * q + a + 24)) : fmax3(pm[a], m3, masked(32 * q + a + 24));
-          }
-        };
+          for (int a = 0; a < 8; ++a) pm[a] = fmax3(pm[a], s[c + a], s[c + a + 8]);
+        const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+        const float m_new = fmaxf(m_run, mx * sl2);
         if (j == 0) {
-          // first tile: the running max must come first
-#pragma unroll
-          for (int c = 0; c < kBlockN / 32; ++c) tmem_ld32(tS + 32u * c, sr + 32 * c);
-          tmem_wait_ld();
-#pragma unroll
-          for (int q = 0; q < kBlockN / 32; ++q) chunk_max(q);
-          const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
-          m_run = (mx == -INFINITY) ? 0.f : mx * sl2;
-#pragma unroll
-          for (int q = 0; q < kBlockN / 32; ++q) exp_chunk(q, -m_run);
+          m_run = (m_new == -INFINITY) ? 0.f : m_new;
         } else {
-          // Later tiles: exponentiate against the running max while the next
-          // 32-column chunk is still being read from tensor memory; check the
-          // new row max afterwards.
-          tmem_ld32(tS, sr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int q = 0; q < kBlockN / 32; ++q) {
-            if (q + 1 < kBlockN / 32) tmem_ld32(tS + 32u * (q + 1), sr + 32 * (q + 1));
-            chunk_max(q);
-            exp_chunk(q, -m_run);
-            if (q + 1 < kBlockN / 32) tmem_wait_ld();
-          }
-          const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
-          const float m_new = mx * sl2;
+          // The rescale touches tensor memory with warp-collective
+          // instructions, so the whole warp takes the branch when any of its
+          // rows needs it; rows that do not keep their max and use alpha = 1.
           const bool need = m_new > m_run + kRescaleThreshold;
           if (__any_sync(0xffffffffu, need)) {
-            // Rare: a row's max grew by more than 2^8.  The whole warp takes
-            // this branch (tensor-memory access is warp-collective); rows that
-            // do not need it keep their max and use alpha = 1.
             const float alpha = need ? ex2_approx(m_run - m_new) : 1.f;
             if (need) {
               l_run *= alpha;
@@ -386,13 +351,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
               tmem_st32(tO + 32u * c, o);
             }
-            // redo P (and its row sum) against the updated max
-            tmem_wait_st();
-#pragma unroll
-            for (int a = 0; a < 4; ++a) ps[a] = 0.f;
-#pragma unroll
-            for (int q = 0; q < kBlockN / 32; ++q) exp_chunk(q, -m_run);
           }
+        }
+        const float neg_m = -m_run;
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int q = 0; q < kBlockN / 32; ++q) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float x0 = fmaf(s[32 * q + 2 * e], sl2, neg_m);
+            const float x1 = fmaf(s[32 * q + 2 * e + 1], sl2, neg_m);
+            const bool poly = (kPolyPairMask >> (e & 7)) & 1u;
+            const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
+            const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+            ps[e & 3] += p0 + p1;
+            pk[e] = pack2<BF16>(p0, p1);
+          }
+          tmem_st16(tS + 16u * q, pk);
         }
         l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         tmem_wait_st();
