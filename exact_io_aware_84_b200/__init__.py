@@ -22,6 +22,7 @@ __all__ = [
     "fa_fwd",
     "fa_bwd",
     "fa_bwd_workspace_size",
+    "fa_bwd_noalloc",
     "fa_status_string",
     "fa_last_device_status",
     "fa_debug_set_wait_limit_ms",
@@ -61,6 +62,8 @@ _SIGNATURES = {
     "fa_bwd_workspace_size": (_sz, [_c_int, _c_int, _c_int, _c_int]),
     "fa_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                         _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _vp]),
+    "fa_bwd_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _vp]),
     "fa_status_string": (ctypes.c_char_p, [_c_int]),
     "fa_last_device_status": (_c_int, [_vp]),
     "fa_debug_set_wait_limit_ms": (_c_int, [_c_int]),
@@ -237,4 +240,31 @@ def fa_bwd(q, k, v, o, do, lse, dq=None, dk=None, dv=None, workspace=None,
                                _stream_handle(stream))
     if st != FA_OK:
         raise FAError(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def fa_bwd_noalloc(q, k, v, o, do, lse, dq=None, dk=None, dv=None, scale: Optional[float] = None,
+                   causal: bool = False, stream=None):
+    """fa_bwd without a workspace argument: the library's fixed 32 MiB scratch
+    is used instead (for callers that cannot allocate device memory).  Calls
+    on one device share that scratch and must not overlap on the GPU."""
+    torch = _torch()
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _check_bhnd(name, t, None if name == "q" else q, allow_f32=(name == "o"))
+    B, H, N, d = q.shape
+    if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B, H, N] tensor")
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_bhnd(name, t, q)
+    st = load_library().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                       lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                       B, H, N, d, float(scale), int(bool(causal)), _dtype_code(q, o),
+                                       _stream_handle(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd_noalloc")
     return dq, dk, dv

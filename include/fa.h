@@ -118,6 +118,29 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
            void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
            float scale, int causal, int dtype, void* stream);
 
+/*
+ * Backward without caller-provided workspace, for callers that cannot
+ * allocate device memory (for example an operator inside a framework whose
+ * allocator owns every device allocation, or a host loop that must not call
+ * cudaMalloc after start-up).  The pages have no counterpart: this is a
+ * library convenience, not part of the method.
+ *   Same arguments and results as fa_bwd, minus workspace/workspace_bytes.
+ *   The scratch fa_bwd needs is taken from a fixed array of 32 MiB
+ *   (33554432 bytes) inside the library's device memory, present on every GPU
+ *   that loads the library until the process exits.  Problems whose
+ *   fa_bwd_workspace_size exceeds it return FA_ERR_WORKSPACE before anything
+ *   runs.  The call allocates nothing.
+ *   The first call on each device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls on a device share the array: calls that overlap on the GPU
+ *   (other streams, other host threads) race and must be serialised by the
+ *   caller.  The array keeps the last call's contents; fa_bwd rewrites every
+ *   part of it that it reads, so no clearing is needed between calls.
+ */
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
+                   int causal, int dtype, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fa_status_string(int status);
 

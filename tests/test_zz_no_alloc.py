@@ -1,0 +1,59 @@
+"""The allocation-free backward entry point (fa_bwd_noalloc) gives the same
+gradients as fa_bwd with caller-allocated workspace.
+
+It is meant for callers that cannot allocate device memory themselves (for
+example a plugin inside a framework that owns every device allocation, or a
+host loop that must not call cudaMalloc after start-up); the scratch lives in
+a fixed array inside the library.  This file is collected last so that a run
+stopping at the first failure has already run every other test, and it
+passes both alone in a fresh process and after the other tests (the scratch
+keeps the previous call's contents, which the backward rewrites each call).
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import exact_io_aware_84_b200 as fa
+from exact_io_aware_84_b200.inputs import Workload, make_inputs
+from parity import TOL_GRAD_REL, rel_fro, to64
+
+pytestmark = pytest.mark.gpu
+
+
+def _call_noalloc(lib, g, o, lse, out, w):
+    return lib.fa_bwd_noalloc(g["q"].data_ptr(), g["k"].data_ptr(), g["v"].data_ptr(), o.data_ptr(),
+                              g["do"].data_ptr(), lse.data_ptr(), out[0].data_ptr(), out[1].data_ptr(),
+                              out[2].data_ptr(), w.B, w.H, w.N, w.d, ctypes.c_float(w.scale), int(w.causal),
+                              0 if w.dtype == "bf16" else 1, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
+@pytest.mark.parametrize("w", [
+    Workload("noalloc_d64", 2, 3, 700, 64, "bf16", True, 0.125, True, seed=21),
+    Workload("noalloc_d128", 1, 4, 513, 128, "bf16", False, 128 ** -0.5, True, seed=22),
+], ids=lambda w: w.name)
+def test_noalloc_matches_fa_bwd_on_two_calls(w):
+    lib = fa.load_library()
+    x = make_inputs(w)
+    g = {k: v.cuda() for k, v in x.items()}
+    o, lse = fa.fa_fwd(g["q"], g["k"], g["v"], scale=w.scale, causal=w.causal)
+    ref = fa.fa_bwd(g["q"], g["k"], g["v"], o, g["do"], lse, scale=w.scale, causal=w.causal)
+    for call in range(2):
+        out = [torch.full_like(g["q"], float("nan")) for _ in range(3)]
+        st = _call_noalloc(lib, g, o, lse, out, w)
+        assert st == fa.FA_OK, fa.fa_status_string(st)
+        torch.cuda.synchronize()
+        assert fa.fa_last_device_status() == fa.FA_OK
+        for name, a, r in zip(("dq", "dk", "dv"), out, ref):
+            e = rel_fro(to64(a), to64(r))
+            assert np.isfinite(to64(a)).all() and e <= TOL_GRAD_REL, (call, name, e)
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    lib = fa.load_library()
+    # 64 heads x 16384 rows x d=128 needs ~0.5 GB of scratch: refused before launch
+    p = ctypes.c_void_p(0x1000)
+    st = lib.fa_bwd_noalloc(p, p, p, p, p, p, p, p, p, 4, 16, 16384, 128, ctypes.c_float(0.1), 0, 0, None)
+    assert st == fa.FA_ERR_WORKSPACE
