@@ -48,6 +48,7 @@ def _args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-target", action="store_true")
+    ap.add_argument("--no-memory", action="store_true")
     return ap.parse_args()
 
 
@@ -322,6 +323,12 @@ def run_native(args):
                         "measured_sustained": value / world / peaks["bf16_tflops_sustained"],
                         "datasheet_2250": value / world / 2250.0},
     }
+    if not args.no_memory and rank == 0:
+        line["memory"] = _memory_vs_n(fa, torch, dev, stream)
+    line["context"] = {
+        "note": "the pages' own figures on other hardware; not targets",
+        "fa2_a100_frac_of_peak": 0.70, "fa1_a100_frac_of_peak": 0.35,
+        "source": "marketmaker.cc, FA2 section (A100 theoretical peak FLOPs)"}
     if not args.no_target and w.name != TARGET_WORKLOAD:
         line["north_star_target"] = _target_fwd(fa, torch, dev, stream, flush, peaks, args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -335,6 +342,34 @@ def run_native(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def _memory_vs_n(fa, torch, dev, stream):
+    """Peak device memory of one forward + backward at d=128, B=2, H=16 for
+    N in {2048, 8192, 16384} (every buffer the call needs: inputs, outputs,
+    workspace), next to the score matrix standard attention would hold
+    (B H N^2 x 2 bytes).  Linear in N: the kernels never store an N x N
+    matrix."""
+    from exact_io_aware_84_b200.metrics import score_matrix_bytes
+    out = {"B": 2, "H": 16, "d": 128, "N": [], "peak_bytes": [], "score_matrix_bytes_bf16": []}
+    for n in (2048, 8192, 16384):
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        torch.cuda.reset_peak_memory_stats(dev)
+        base = torch.cuda.memory_allocated(dev)
+        shape = (2, 16, n, 128)
+        q, k, v, do = (torch.randn(shape, device=dev, dtype=torch.bfloat16) for _ in range(4))
+        o, lse = fa.fa_fwd(q, k, v, stream=stream)
+        fa.fa_bwd(q, k, v, o, do, lse, stream=stream)
+        torch.cuda.synchronize()
+        out["N"].append(n)
+        out["peak_bytes"].append(int(torch.cuda.max_memory_allocated(dev) - base))
+        out["score_matrix_bytes_bf16"].append(score_matrix_bytes(2, 16, n, 2))
+        del q, k, v, do, o, lse
+    per_n = [b / n for b, n in zip(out["peak_bytes"], out["N"])]
+    out["bytes_per_token"] = per_n
+    out["linear_in_n"] = max(per_n) / min(per_n) < 1.05
+    return out
 
 
 def _target_fwd(fa, torch, dev, stream, flush, peaks, args):

@@ -53,20 +53,22 @@ struct BwdLayout {
   static constexpr int kStage = BR * D * 4;        // fp32 dQ staging bytes
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kKOff + kKV;
-  static constexpr int kQOff = kVOff + kKV;        // [2] stages
-  static constexpr int kDOOff = kQOff + 2 * kQT;   // [2] stages
-  static constexpr int kDSOff = kDOOff + 2 * kQT;
+  static constexpr int kStages = 3;               // Q / dO / LSE / D ring depth
+  static constexpr int kQOff = kVOff + kKV;        // [kStages]
+  static constexpr int kDOOff = kQOff + kStages * kQT;
+  static constexpr int kDSOff = kDOOff + kStages * kQT;
   static constexpr int kStgOff = kDSOff + kDS;
-  static constexpr int kVecOff = kStgOff + kStage;  // [2] stages x (lse2[BR], dvec[BR])
+  static constexpr int kVecOff = kStgOff + kStage;  // [kStages] x (lse2[BR], dvec[BR])
   static constexpr int kVecStage = 2 * BR * 4;
-  static constexpr int kBarOff = kVecOff + 2 * kVecStage;
+  static constexpr int kBarOff = kVecOff + kStages * kVecStage;
   // barriers
   static constexpr int kKVFull = 0, kKVEmpty = 1;
-  static constexpr int kQFull = 2;   // [2]
-  static constexpr int kQEmpty = 4;  // [2]
-  static constexpr int kSFull = 6, kDPFull = 7, kPFull = 8, kDSFull = 9, kDSEmpty = 10;
-  static constexpr int kDQFull = 11, kDQEmpty = 12, kAccFull = 13, kAccEmpty = 14, kDrain = 15;
-  static constexpr int kNumBars = 16;
+  static constexpr int kQFull = 2;                 // [kStages]
+  static constexpr int kQEmpty = kQFull + kStages;  // [kStages]
+  static constexpr int kSFull = kQEmpty + kStages, kDPFull = kSFull + 1, kPFull = kSFull + 2;
+  static constexpr int kDSFull = kSFull + 3, kDSEmpty = kSFull + 4, kDQFull = kSFull + 5;
+  static constexpr int kDQEmpty = kSFull + 6, kAccFull = kSFull + 7, kAccEmpty = kSFull + 8, kDrain = kSFull + 9;
+  static constexpr int kNumBars = kDrain + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -149,7 +151,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(BAR(L::kKVFull), 1);
     mbar_init(BAR(L::kKVEmpty), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < L::kStages; ++s) {
       mbar_init(BAR(L::kQFull + s), 1);
       mbar_init(BAR(L::kQEmpty + s), 1);
     }
@@ -199,7 +201,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tma_load_3d(base + L::kVOff + c * (kBlockN * 128), &tmV, BAR(L::kKVFull), c * 64, bu.jk * kBlockN, bu.bh, pol_kv);
         }
         for (int i = bu.i0; i <= bu.i1; ++i, ++q_iter) {
-          const uint32_t st = q_iter & 1, use = q_iter >> 1;
+          const uint32_t st = q_iter % L::kStages, use = q_iter / L::kStages;
           if (use > 0 && !mbar_wait(BAR(L::kQEmpty + st), (use - 1) & 1, wc)) { ok = false; break; }
           const uint32_t fb = BAR(L::kQFull + st);
           mbar_arrive_expect_tx(fb, 2 * L::kQT + L::kVecStage);
@@ -215,8 +217,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       if (!ok) {
         if (unit_iter > 0) mbar_wait_drain(BAR(L::kKVFull), (unit_iter - 1) & 1, p.wait_limit_ns);
-        for (uint32_t s = 0; s < 2; ++s) {
-          const uint32_t issued = q_iter / 2 + (s < (q_iter & 1) ? 1u : 0u);
+        for (uint32_t s = 0; s < (uint32_t)L::kStages; ++s) {
+          const uint32_t issued = q_iter / L::kStages + (s < q_iter % L::kStages ? 1u : 0u);
           if (issued > 0) mbar_wait_drain(BAR(L::kQFull + s), (issued - 1) & 1, p.wait_limit_ns);
         }
       }
@@ -236,8 +238,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t sK = base + L::kKOff, sV = base + L::kVOff;
         // S^T for the first query tile
         {
-          const uint32_t st = q_iter & 1;
-          if (!mbar_wait(BAR(L::kQFull + st), (q_iter >> 1) & 1, wc)) { ok = false; break; }
+          const uint32_t st = q_iter % L::kStages;
+          if (!mbar_wait(BAR(L::kQFull + st), (q_iter / L::kStages) & 1, wc)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sQ = base + L::kQOff + st * L::kQT;
 #pragma unroll
@@ -246,7 +248,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_commit(BAR(L::kSFull));
         }
         for (int i = bu.i0; i <= bu.i1; ++i, ++q_iter) {
-          const uint32_t st = q_iter & 1;
+          const uint32_t st = q_iter % L::kStages;
           const uint32_t sQ = base + L::kQOff + st * L::kQT;
           const uint32_t sDO = base + L::kDOOff + st * L::kQT;
           const uint32_t first = (i == bu.i0);
@@ -266,8 +268,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mma_ts(tmem + L::kColDV, tmem + L::kColS + 8u * ks, mnmaj<BR>(sDO, ks), idesc_acc, (!first || ks > 0) ? 1u : 0u);
           // S^T for the next query tile (the S region's P^T was consumed by dV above)
           if (i < bu.i1) {
-            const uint32_t st1 = (q_iter + 1) & 1;
-            if (!mbar_wait(BAR(L::kQFull + st1), ((q_iter + 1) >> 1) & 1, wc)) { ok = false; break; }
+            const uint32_t st1 = (q_iter + 1) % L::kStages;
+            if (!mbar_wait(BAR(L::kQFull + st1), ((q_iter + 1) / L::kStages) & 1, wc)) { ok = false; break; }
             tc_fence_after();
             const uint32_t sQ1 = base + L::kQOff + st1 * L::kQT;
 #pragma unroll
@@ -319,8 +321,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int key = bu.jk * kBlockN + key_in;
       const bool key_ok = key < p.N;
       for (int i = bu.i0; i <= bu.i1; ++i, ++q_iter) {
-        const uint32_t st = q_iter & 1;
-        ok = warp_all(mbar_wait(BAR(L::kQFull + st), (q_iter >> 1) & 1, wc));
+        const uint32_t st = q_iter % L::kStages;
+        ok = warp_all(mbar_wait(BAR(L::kQFull + st), (q_iter / L::kStages) & 1, wc));
         if (!ok) break;
         const float* lse2 = reinterpret_cast<const float*>(gbase + L::kVecOff + st * L::kVecStage);
         const float* dvec = lse2 + BR;
@@ -359,12 +361,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = warp_all(ds_cnt == 0 || mbar_wait(BAR(L::kDSEmpty), (ds_cnt - 1) & 1, wc));
         if (!ok) break;
         ++ds_cnt;
-        uint32_t dsk[BR / 2];
+        // dS^T chunk by chunk (32 queries): into tensor memory for the dK MMA
+        // and into the SW128 shared tile [key][query] for the dQ MMA.  In
+        // the shared tile, column block cb holds queries 64cb..64cb+63 and
+        // 16-byte chunk ch of row `key_in` lives at position ch ^ (key_in & 7).
+        uint8_t* ds_tile = gbase + L::kDSOff;
 #pragma unroll
         for (int c = 0; c < BR / 32; ++c) {
           uint32_t r[32];
           tmem_ld32(tDP + 32u * c, r);
           tmem_wait_ld();
+          uint32_t dsk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int qa = 32 * c + 2 * e;
@@ -380,21 +387,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             const float ds0 = p0 * (__uint_as_float(r[2 * e]) - dvec[qa]);
             const float ds1 = p1 * (__uint_as_float(r[2 * e + 1]) - dvec[qa + 1]);
-            dsk[16 * c + e] = pack2<BF16>(ds0, ds1);
+            dsk[e] = pack2<BF16>(ds0, ds1);
           }
-        }
+          // dS^T chunk c goes to columns [16c, 16c+16) of the dP^T region:
+          // those belong to dP^T chunk c/2, already read; the chunks still to
+          // be read start at column 32(c+1) > 16c + 16.
+          tmem_st16(tDP + 16u * c, dsk);
+          const int cb = c >> 1;
 #pragma unroll
-        for (int c = 0; c < BR / 32; ++c) tmem_st16(tDP + 16u * c, dsk + 16 * c);
-        // dS^T row (this key) into the SW128 shared tile [key][query]:
-        // column block cb holds queries 64cb..64cb+63; 16-byte chunk ch of
-        // row `key_in` lives at chunk position ch ^ (key_in & 7).
-        uint8_t* ds_tile = gbase + L::kDSOff;
-#pragma unroll
-        for (int cb = 0; cb < BR / 64; ++cb) {
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            uint4 val = make_uint4(dsk[32 * cb + 4 * ch], dsk[32 * cb + 4 * ch + 1], dsk[32 * cb + 4 * ch + 2],
-                                   dsk[32 * cb + 4 * ch + 3]);
+          for (int h = 0; h < 4; ++h) {
+            const int ch = (c & 1) * 4 + h;
+            uint4 val = make_uint4(dsk[4 * h], dsk[4 * h + 1], dsk[4 * h + 2], dsk[4 * h + 3]);
             *reinterpret_cast<uint4*>(ds_tile + cb * (kBlockN * 128) + key_in * 128 + ((ch ^ (key_in & 7)) * 16)) = val;
           }
         }
@@ -421,41 +424,56 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         // 64 fp32 columns per lane: d=64 -> lane = query, cols = dims;
         //                           d=128 -> lane = dim, cols = queries.
-        uint32_t v[64];
-        tmem_ld32(tmem + lane_off + L::kColDQ, v);
-        tmem_ld32(tmem + lane_off + L::kColDQ + 32, v + 32);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(BAR(L::kDQEmpty));
-        // the previous bulk reduce must have finished reading the staging tile
-        if (t == 0) bulk_wait_read0();
-        named_bar_sync(1, 128);
         if (D == 64) {
-          // row t of [128 queries][64 dims].  Lanes write different 16-byte
-          // chunks at the same time (chunk (e + t) mod 16 at step e) to spread
-          // shared-memory banks; the registers are first rotated by t chunks
-          // with a static barrel shifter so that no array is indexed by a
-          // lane-dependent value.
-          const int rot = t & 15;
+          // lane t = query t, 64 fp32 columns = dims, staged as row t of the
+          // [128 queries][64 dims] tile.  Each 32-column half is read,
+          // scaled and written with its eight 16-byte chunks rotated by t mod 8
+          // (positions (e + t) mod 8 at step e), so lanes spread over all
+          // banks; the rotation is a static barrel shift of the registers.
+          uint32_t v[32];
 #pragma unroll
-          for (int b = 1; b < 16; b <<= 1) {
-            if (rot & b) {
-              uint32_t tmp[64];
+          for (int h = 0; h < 2; ++h) {
+            tmem_ld32(tmem + lane_off + L::kColDQ + 32u * h, v);
+            tmem_wait_ld();
+            if (h == 1) {
+              tc_fence_before();
+              mbar_arrive(BAR(L::kDQEmpty));
+            }
+            if (h == 0) {
+              // the previous bulk reduce must have finished reading the tile
+              if (t == 0) bulk_wait_read0();
+              named_bar_sync(1, 128);
+            }
+            const int rot = t & 7;
 #pragma unroll
-              for (int e = 0; e < 64; ++e) tmp[e] = v[(e + 4 * b) & 63];
+            for (int b = 1; b < 8; b <<= 1) {
+              if (rot & b) {
+                uint32_t tmp[32];
 #pragma unroll
-              for (int e = 0; e < 64; ++e) v[e] = tmp[e];
+                for (int e = 0; e < 32; ++e) tmp[e] = v[(e + 4 * b) & 31];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = tmp[e];
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int ch = 8 * h + ((e + t) & 7);
+              float4 f = make_float4(__uint_as_float(v[4 * e]) * p.scale, __uint_as_float(v[4 * e + 1]) * p.scale,
+                                     __uint_as_float(v[4 * e + 2]) * p.scale, __uint_as_float(v[4 * e + 3]) * p.scale);
+              *reinterpret_cast<float4*>(stage + t * 64 + 4 * ch) = f;
             }
           }
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int ch = (e + t) & 15;
-            float4 f = make_float4(__uint_as_float(v[4 * e]) * p.scale, __uint_as_float(v[4 * e + 1]) * p.scale,
-                                   __uint_as_float(v[4 * e + 2]) * p.scale, __uint_as_float(v[4 * e + 3]) * p.scale);
-            *reinterpret_cast<float4*>(stage + t * 64 + 4 * ch) = f;
-          }
         } else {
-          // column t of [64 queries][128 dims]
+          // lane t = dim t, 64 fp32 columns = queries: column t of the
+          // [64 queries][128 dims] tile (consecutive lanes, consecutive words)
+          uint32_t v[64];
+          tmem_ld32(tmem + lane_off + L::kColDQ, v);
+          tmem_ld32(tmem + lane_off + L::kColDQ + 32, v + 32);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(BAR(L::kDQEmpty));
+          if (t == 0) bulk_wait_read0();
+          named_bar_sync(1, 128);
 #pragma unroll
           for (int q = 0; q < 64; ++q) stage[q * 128 + t] = __uint_as_float(v[q]) * p.scale;
         }

@@ -34,12 +34,19 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only if max grows > 2^8
 // Which of the 8 element pairs in every 16 columns take exp2 on the FMA pipe
-// (exp2_poly) instead of the MUFU unit: bit k set = pair k.  Balances the
-// two pipes; the MUFU alone caps the softmax at 16 exponentials/clock/SM.
-#ifndef FA_FWD_POLY_PAIR_MASK
-#define FA_FWD_POLY_PAIR_MASK 0x00
+// (exp2_poly) instead of the MUFU unit: bit k set = pair k.  The MUFU alone
+// caps the softmax at 16 exponentials/clock/SM; at d = 64 each exponential
+// carries half the MMA work of d = 128, so only d = 64 is MUFU-bound.
+#ifndef FA_FWD_POLY_PAIR_MASK_D64
+#define FA_FWD_POLY_PAIR_MASK_D64 0x00
 #endif
-constexpr uint32_t kPolyPairMask = FA_FWD_POLY_PAIR_MASK;
+#ifndef FA_FWD_POLY_PAIR_MASK_D128
+#define FA_FWD_POLY_PAIR_MASK_D128 0x00
+#endif
+template <int D>
+constexpr uint32_t poly_pair_mask() {
+  return D == 64 ? FA_FWD_POLY_PAIR_MASK_D64 : FA_FWD_POLY_PAIR_MASK_D128;
+}
 // Register split.  Launch: 384 threads x 168 registers.  Warp w runs on SM
 // sub-partition w % 4, which therefore holds warps {k, k+4, k+8}: two softmax
 // warps and one warp of the producer/MMA warpgroup.  Each sub-partition's
@@ -49,10 +56,14 @@ constexpr int kRegsSoftmax = 216;
 constexpr int kRegsOther = 72;
 static_assert(2 * kRegsSoftmax + kRegsOther <= 3 * kLaunchRegs, "register split exceeds a sub-partition's pool");
 
+#ifndef FA_FWD_SLOTS_D128
+#define FA_FWD_SLOTS_D128 4
+#endif
+
 template <int D>
 struct FwdLayout {
   static constexpr int kTile = kBlockM * D * 2;  // bytes of one 128 x D 16-bit tile
-  static constexpr int kSlots = (D == 128) ? 4 : 8;
+  static constexpr int kSlots = (D == 128) ? FA_FWD_SLOTS_D128 : 8;  // K/V ring depth (tiles)
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTile;
   static constexpr int kBarOff = kKVOff + kSlots * kTile;
@@ -73,6 +84,7 @@ struct FwdLayout {
   // tensor-memory columns
   static constexpr uint32_t kColS0 = 0;
   static constexpr uint32_t kColO0 = 256;
+  static_assert(kAlloc <= 232448, "shared memory overflow");
 };
 
 struct UnitInfo {
@@ -221,11 +233,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint32_t kv_base = kv_iter;
         for (int j = 0; j <= ui.nmax && ok; ++j) {
           const uint32_t k_idx = kv_base + 2 * j, v_idx = kv_base + 2 * (j - 1) + 1;
-          if (j < ui.nmax) {
-            if (!mbar_wait(BAR(L::kKVFull + k_idx % L::kSlots), (k_idx / L::kSlots) & 1, wc)) { ok = false; break; }
-            tc_fence_after();
-          }
-          bool v_ready = false;
+          bool v_ready = false, k_ready = false;
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
             const int nbt = ui.nb(t);
@@ -252,6 +260,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               if (j == nbt) tc_commit(BAR(L::kOFull + t));
             }
             if (j < nbt) {
+              // K_j is waited for only here, after the PV MMAs of block j-1
+              // (which do not need it) have been issued.
+              if (!k_ready) {
+                ok = mbar_wait(BAR(L::kKVFull + k_idx % L::kSlots), (k_idx / L::kSlots) & 1, wc);
+                k_ready = true;
+                if (!ok) continue;
+                tc_fence_after();
+              }
               // S_t = Q_t K_j^T
               const uint32_t qt = base + L::kQOff + t * L::kTile;
               const uint32_t kt = base + L::kKVOff + (k_idx % L::kSlots) * L::kTile;
@@ -263,10 +279,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
           if (!ok) break;
           if (j == ui.nmax - 1) tc_commit(BAR(L::kQEmpty));
-          if (j >= 1) {
-            tc_commit(BAR(L::kKVEmpty + (kv_base + 2 * (j - 1)) % L::kSlots));
-            tc_commit(BAR(L::kKVEmpty + v_idx % L::kSlots));
-          }
+          // Release K_j as soon as the S MMAs of block j are issued (they are
+          // its last readers) and V_{j-1} after the PV MMAs of block j-1; the
+          // producer can then refill the slots about one block ahead.
+          if (j < ui.nmax) tc_commit(BAR(L::kKVEmpty + k_idx % L::kSlots));
+          if (j >= 1) tc_commit(BAR(L::kKVEmpty + v_idx % L::kSlots));
         }
         kv_iter = kv_base + 2 * ui.nmax;
         o_uses0 += 1;
@@ -362,7 +379,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int e = 0; e < 16; ++e) {
             const float x0 = fmaf(s[32 * q + 2 * e], sl2, neg_m);
             const float x1 = fmaf(s[32 * q + 2 * e + 1], sl2, neg_m);
-            const bool poly = (kPolyPairMask >> (e & 7)) & 1u;
+            const bool poly = (poly_pair_mask<D>() >> (e & 7)) & 1u;
             const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
             const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
             ps[e & 3] += p0 + p1;
