@@ -437,18 +437,34 @@ def _e2e(fa, torch, w, x, dev, stream, flops, world, args):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
+def kernel_sources_hash():
+    """sha1 prefix of the CUDA sources (file names and contents, sorted)."""
+    import glob
+    import hashlib
+    h = hashlib.sha1()
+    for f in sorted(glob.glob(os.path.join(ROOT, "exact_io_aware_84_b200", "csrc", "*"))):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(os.path.basename(f).encode())
+            with open(f, "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def _ncu_traffic(workload_name, kernel_name):
-    """DRAM bytes per launch from a committed ncu summary, when one exists for
-    this workload and the current kernels (else null)."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch of the dominant kernel group, from the committed
+    ncu summary for this workload (profiles/traffic_<workload>.md), but only
+    while the kernel sources are the ones that summary was captured from;
+    otherwise null."""
+    import re
+    path = os.path.join(ROOT, "profiles", f"traffic_{workload_name}.md")
     if not os.path.exists(path):
         return None
-    try:
-        with open(path) as f:
-            d = json.load(f)
-        return d.get(workload_name, {}).get("dram_bytes_per_launch")
-    except Exception:
+    text = open(path).read()
+    m_hash = re.search(r"Kernel sources: `([0-9a-f]+)`", text)
+    m_val = re.search(r"bench\.py traffic key: " + re.escape(workload_name) + r"=(\d+)", text)
+    if not m_hash or not m_val or m_hash.group(1) != kernel_sources_hash():
         return None
+    return int(m_val.group(1))
 
 
 def main():
