@@ -11,4 +11,6 @@ from .attention import (  # noqa: F401
     attn_bwd_ref,
     online_fwd_ref,
     fa1_fwd_ref,
+    gqa_fwd_ref,
+    gqa_bwd_ref,
 )

@@ -33,6 +33,13 @@ What it computes (all in float64, on whatever arrays it is handed):
   are reconstructed from its prose, which says that whenever a block raises
   the running maximum the output accumulated so far is multiplied by
   e^{m^(j-1) - m^(j)}).
+* ``gqa_fwd_ref`` / ``gqa_bwd_ref`` -- grouped-query attention: H query heads
+  share Hkv key/value heads, query head h reading key/value head
+  h // (H / Hkv).  The forward is the definition above with K and V repeated
+  per group; the gradient of K and V is the chain rule of that repetition
+  (the per-query-head gradients summed over the group).  The delect.ru
+  glossary ("What is confirmed") notes that the attention computation does
+  not change the number of key/value heads: grouping is orthogonal to it.
 * ``fa1_fwd_ref`` -- the per-step-normalised loop of the marketmaker.cc
   section "The Flash Attention algorithm" (query blocks outer, key/value blocks
   inner, O normalised by the running sum after every block).
@@ -60,6 +67,8 @@ __all__ = [
     "attn_bwd_ref",
     "online_fwd_ref",
     "fa1_fwd_ref",
+    "gqa_fwd_ref",
+    "gqa_bwd_ref",
 ]
 
 
@@ -268,3 +277,30 @@ def fa1_fwd_ref(q, k, v, scale, causal=False, block_r=128, block_c=128):
         lse_all[rows] = (m + np.log(np.where(l > 0, l, 1.0)))[:, 0]
     return o_all, lse_all
 
+
+
+def _repeat_kv(x, group):
+    """[B, Hkv, N, d] -> [B, Hkv*group, N, d], each key/value head repeated
+    for the `group` consecutive query heads that read it."""
+    return np.repeat(_f64(x), group, axis=1)
+
+
+def gqa_fwd_ref(q, k, v, scale, causal=False, row_chunk=1024):
+    """Grouped-query forward: q [B, H, N, d]; k, v [B, Hkv, N, d]."""
+    H, Hkv = np.asarray(q).shape[1], np.asarray(k).shape[1]
+    assert H % Hkv == 0
+    g = H // Hkv
+    return attn_fwd_ref(q, _repeat_kv(k, g), _repeat_kv(v, g), scale, causal, row_chunk)
+
+
+def gqa_bwd_ref(q, k, v, do, scale, causal=False, row_chunk=1024):
+    """Grouped-query gradient: dQ per query head; dK, dV summed over the
+    query heads of each group."""
+    q = _f64(q)
+    B, H = q.shape[:2]
+    Hkv = np.asarray(k).shape[1]
+    assert H % Hkv == 0
+    g = H // Hkv
+    dq, dk, dv = attn_bwd_ref(q, _repeat_kv(k, g), _repeat_kv(v, g), do, scale, causal, row_chunk)
+    n, d = dk.shape[-2:]
+    return dq, dk.reshape(B, Hkv, g, n, d).sum(2), dv.reshape(B, Hkv, g, n, d).sum(2)

@@ -23,7 +23,7 @@ import torch
 
 from oracle import (attn_bwd_ref, attn_fwd_ref, attn_fwd_rows_ref,
                     attn_probs_ref, attn_scores_ref, fa1_fwd_ref,
-                    online_fwd_ref)
+                    gqa_bwd_ref, gqa_fwd_ref, online_fwd_ref)
 from exact_io_aware_84_b200.metrics import score_matrix_bytes
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -340,3 +340,61 @@ def test_score_matrix_memory_worked_examples():
         got = score_matrix_bytes(int(B), int(H), int(s), int(e))
         assert got == int(expect)
         assert abs(got / 1e9 - float(page_gb)) <= float(tol) * float(page_gb)
+
+
+# ------------------------------------------------------- grouped-query heads
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_forward_brute_force(causal):
+    # 4 query heads over 2 key/value heads: query head h reads kv head h // 2
+    r = _rng(40 + causal)
+    q = r.standard_normal((1, 4, 6, 3))
+    k = r.standard_normal((1, 2, 6, 3))
+    v = r.standard_normal((1, 2, 6, 2))
+    o, lse = gqa_fwd_ref(q, k, v, 0.7, causal)
+    for h in range(4):
+        ob, lb = _brute_fwd(q[0, h], k[0, h // 2], v[0, h // 2], 0.7, causal)
+        np.testing.assert_allclose(o[0, h], ob, atol=1e-14)
+        np.testing.assert_allclose(lse[0, h], lb, atol=1e-14)
+
+
+def test_gqa_group_of_one_is_multi_head():
+    r = _rng(42)
+    q, k, v, do = (r.standard_normal((2, 3, 9, 4)) for _ in range(4))
+    for a, b in zip(gqa_fwd_ref(q, k, v, 0.5, True), attn_fwd_ref(q, k, v, 0.5, True)):
+        np.testing.assert_array_equal(a, b)
+    for a, b in zip(gqa_bwd_ref(q, k, v, do, 0.5, True), attn_bwd_ref(q, k, v, do, 0.5, True)):
+        np.testing.assert_array_equal(a, b)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_gradient_matches_finite_differences(causal):
+    # the shared key/value heads receive gradient from every query head of
+    # their group: central differences of L = sum(dO * O) over all heads
+    r = _rng(43 + causal)
+    H, Hkv, n, d = 4, 2, 5, 3
+    q = r.standard_normal((1, H, n, d))
+    k = r.standard_normal((1, Hkv, n, d))
+    v = r.standard_normal((1, Hkv, n, d))
+    do = r.standard_normal((1, H, n, d))
+    scale, h_step = 0.6, 1e-6
+
+    def loss():
+        tot = 0.0
+        for hh in range(H):
+            o, _ = _brute_fwd(q[0, hh], k[0, hh // 2], v[0, hh // 2], scale, causal)
+            tot += float(np.sum(do[0, hh] * o))
+        return tot
+
+    dq, dk, dv = gqa_bwd_ref(q, k, v, do, scale, causal)
+    for x, ana in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + h_step
+            lp = loss()
+            x[idx] = old - h_step
+            lm = loss()
+            x[idx] = old
+            num[idx] = (lp - lm) / (2 * h_step)
+        np.testing.assert_allclose(ana, num, rtol=1e-5, atol=1e-7)
