@@ -23,6 +23,8 @@ __all__ = [
     "fa_bwd",
     "fa_bwd_workspace_size",
     "fa_bwd_noalloc",
+    "fa_fwd_gqa",
+    "fa_bwd_gqa",
     "fa_status_string",
     "fa_last_device_status",
     "fa_debug_set_wait_limit_ms",
@@ -62,6 +64,10 @@ _SIGNATURES = {
     "fa_bwd_workspace_size": (_sz, [_c_int, _c_int, _c_int, _c_int]),
     "fa_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                         _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _vp]),
+    "fa_fwd_gqa": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int,
+                            _c_int, _vp]),
+    "fa_bwd_gqa": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                            _c_int, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _vp]),
     "fa_bwd_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _vp]),
     "fa_status_string": (ctypes.c_char_p, [_c_int]),
@@ -267,4 +273,75 @@ def fa_bwd_noalloc(q, k, v, o, do, lse, dq=None, dk=None, dv=None, scale: Option
                                        _stream_handle(stream))
     if st != FA_OK:
         raise FAError(st, "fa_bwd_noalloc")
+    return dq, dk, dv
+
+
+def _check_kv(name, t, q):
+    _check_bhnd(name, t)
+    if t.dtype != q.dtype or t.device != q.device or t.shape[0] != q.shape[0] or t.shape[2:] != q.shape[2:]:
+        raise ValueError(f"{name} must be [B, Hkv, N, d] with q's B, N, d, dtype and device")
+    if q.shape[1] % t.shape[1] != 0:
+        raise ValueError(f"q's {q.shape[1]} heads are not a multiple of {name}'s {t.shape[1]}")
+
+
+def fa_fwd_gqa(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: bool = False, stream=None,
+               o_fp32: bool = False):
+    """Grouped-query forward: q [B, H, N, d]; k, v [B, Hkv, N, d] with H % Hkv == 0."""
+    torch = _torch()
+    _check_bhnd("q", q)
+    _check_kv("k", k, q)
+    _check_kv("v", v, q)
+    if v.shape != k.shape:
+        raise ValueError("k and v must have the same shape")
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    if o is None:
+        o = torch.empty(q.shape, dtype=torch.float32 if o_fp32 else q.dtype, device=q.device)
+    else:
+        _check_bhnd("o", o, q, allow_f32=True)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    elif lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B, H, N] tensor")
+    st = load_library().fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                   B, H, Hkv, N, d, float(scale), int(bool(causal)), _dtype_code(q, o),
+                                   _stream_handle(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd_gqa")
+    return o, lse
+
+
+def fa_bwd_gqa(q, k, v, o, do, lse, dq=None, dk=None, dv=None, workspace=None,
+               scale: Optional[float] = None, causal: bool = False, stream=None):
+    """Grouped-query backward: dQ per query head; dK, dV summed over each group."""
+    torch = _torch()
+    _check_bhnd("q", q)
+    _check_kv("k", k, q)
+    _check_kv("v", v, q)
+    _check_bhnd("o", o, q, allow_f32=True)
+    _check_bhnd("do", do, q)
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B, H, N] tensor")
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_bhnd("dq", dq, q)
+    _check_kv("dk", dk, q)
+    _check_kv("dv", dv, q)
+    need = fa_bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = load_library().fa_bwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                   lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                   workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                   B, H, Hkv, N, d, float(scale), int(bool(causal)), _dtype_code(q, o),
+                                   _stream_handle(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd_gqa")
     return dq, dk, dv

@@ -155,11 +155,12 @@ int fa_debug_exp2_poly(const float* x, float* y, int n, void* stream) {
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
-           float scale, int causal, int dtype, void* stream) {
+static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                    int N, int d, float scale, int causal, int dtype, void* stream) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   int st = check_common(B, H, N, d, scale, dtype);
   if (st != FA_OK) return st;
+  if (Hkv <= 0 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return FA_ERR_MISALIGNED;
   DeviceInfo di;
@@ -169,14 +170,16 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   const int bh = B * H;
   CUtensorMap tq, tk, tv;
   if (encode_tile_map(&tq, q, bh, N, d, bf16, kBlockM) != FA_OK ||
-      encode_tile_map(&tk, k, bh, N, d, bf16, kBlockN) != FA_OK ||
-      encode_tile_map(&tv, v, bh, N, d, bf16, kBlockN) != FA_OK)
+      encode_tile_map(&tk, k, B * Hkv, N, d, bf16, kBlockN) != FA_OK ||
+      encode_tile_map(&tv, v, B * Hkv, N, d, bf16, kBlockN) != FA_OK)
     return FA_ERR_CUDA;
   FwdParams p{};
   p.o = o;
   p.lse = lse;
   p.N = N;
   p.bh = bh;
+  p.H = H;
+  p.group = H / Hkv;
   p.n_kv = (N + kBlockN - 1) / kBlockN;
   p.n_pairs = (N + 2 * kBlockM - 1) / (2 * kBlockM);
   p.n_units = bh * p.n_pairs;
@@ -189,6 +192,16 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+           float scale, int causal, int dtype, void* stream) {
+  return fwd_impl(q, k, v, o, lse, B, H, H, N, d, scale, causal, dtype, stream);
+}
+
+int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
+               int d, float scale, int causal, int dtype, void* stream) {
+  return fwd_impl(q, k, v, o, lse, B, H, Hkv, N, d, scale, causal, dtype, stream);
+}
+
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   if (check_common(B, H, N, d, 1.0f, FA_BF16) != FA_OK) return 0;
   const size_t n_pad = ((size_t)N + kBlockN - 1) / kBlockN * kBlockN;
@@ -197,12 +210,13 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return up(bh * n_pad * d * sizeof(float)) + 2 * up(bh * n_pad * sizeof(float));
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
-           void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
-           float scale, int causal, int dtype, void* stream) {
+static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                    const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B,
+                    int H, int Hkv, int N, int d, float scale, int causal, int dtype, void* stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   int st = check_common(B, H, N, d, scale, dtype);
   if (st != FA_OK) return st;
+  if (Hkv <= 0 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
       !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return FA_ERR_MISALIGNED;
@@ -225,7 +239,8 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   p.n_kv = (N + kBlockN - 1) / kBlockN;
   p.n_pad = p.n_kv * kBlockN;
   p.bh = bh;
-  p.n_units = bh * p.n_kv;
+  p.group = H / Hkv;
+  p.n_units = B * Hkv * p.n_kv;
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
   p.wait_limit_ns = wait_limit_ns();
@@ -238,13 +253,27 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   CUtensorMap tq, tk, tv, tdo;
   const int q_rows = (d == 64) ? 128 : 64;  // backward query tile (see fa_bwd_sm100.cu)
   if (encode_tile_map(&tq, q, bh, N, d, bf16, q_rows) != FA_OK ||
-      encode_tile_map(&tk, k, bh, N, d, bf16, kBlockN) != FA_OK ||
-      encode_tile_map(&tv, v, bh, N, d, bf16, kBlockN) != FA_OK ||
+      encode_tile_map(&tk, k, B * Hkv, N, d, bf16, kBlockN) != FA_OK ||
+      encode_tile_map(&tv, v, B * Hkv, N, d, bf16, kBlockN) != FA_OK ||
       encode_tile_map(&tdo, dout, bh, N, d, bf16, q_rows) != FA_OK)
     return FA_ERR_CUDA;
   const int grid = p.n_units < di.sms ? p.n_units : di.sms;
   cudaError_t e = launch_bwd(d, bf16, o32, causal != 0, tq, tk, tv, tdo, p, grid, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+           void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+           float scale, int causal, int dtype, void* stream) {
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, H, N, d, scale, causal,
+                  dtype, stream);
+}
+
+int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+               void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int N,
+               int d, float scale, int causal, int dtype, void* stream) {
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, N, d, scale, causal,
+                  dtype, stream);
 }
 
 }  // extern "C"

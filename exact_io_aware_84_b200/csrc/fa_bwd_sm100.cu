@@ -83,22 +83,36 @@ struct BwdLayout {
 };
 
 struct BUnit {
-  int bh, jk, i0, i1;  // key tile jk; query tiles i0..i1 (inclusive)
+  int kvbh;   // batch * Hkv + key/value head
+  int qbh0;   // batch * H + first query head of the group
+  int jk;     // key tile
+  int i0;     // first query tile (causal: the diagonal one)
+  int n_i;    // query tiles per query head
+  int n_it;   // iterations: group x n_i (query head major)
+  __device__ __forceinline__ int qbh(int it) const { return qbh0 + it / n_i; }
+  __device__ __forceinline__ int qtile(int it) const { return i0 + it % n_i; }
 };
 
+// Unit = (batch, key/value head, 128-key tile).  Its iterations run over the
+// query heads that share the key/value head (grouped-query attention; one
+// head when H = Hkv) and, for each, over the query tiles that see the key
+// tile, so dK and dV accumulate over the whole group in tensor memory.
 template <int D, bool CAUSAL>
 __device__ __forceinline__ BUnit decode_bunit(int u, const BwdParams& p) {
   constexpr int BR = BwdLayout<D>::BR;
   BUnit r;
+  const int bhkv = p.bh / p.group;  // B * Hkv
   if (CAUSAL) {  // key tile 0 has the most query tiles: longest first
-    r.jk = u / p.bh;
-    r.bh = u % p.bh;
+    r.jk = u / bhkv;
+    r.kvbh = u % bhkv;
   } else {       // neighbouring CTAs share a head (Q / dO reuse in L2)
     r.jk = u % p.n_kv;
-    r.bh = u / p.n_kv;
+    r.kvbh = u / p.n_kv;
   }
+  r.qbh0 = r.kvbh * p.group;  // (b * Hkv + hkv) * group = b * H + hkv * group
   r.i0 = CAUSAL ? (r.jk * kBlockN) / BR : 0;
-  r.i1 = (p.N + BR - 1) / BR - 1;
+  r.n_i = (p.N + BR - 1) / BR - r.i0;
+  r.n_it = r.n_i * p.group;
   return r;
 }
 
@@ -197,20 +211,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_arrive_expect_tx(BAR(L::kKVFull), 2 * L::kKV);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(base + L::kKOff + c * (kBlockN * 128), &tmK, BAR(L::kKVFull), c * 64, bu.jk * kBlockN, bu.bh, pol_kv);
-          tma_load_3d(base + L::kVOff + c * (kBlockN * 128), &tmV, BAR(L::kKVFull), c * 64, bu.jk * kBlockN, bu.bh, pol_kv);
+          tma_load_3d(base + L::kKOff + c * (kBlockN * 128), &tmK, BAR(L::kKVFull), c * 64, bu.jk * kBlockN, bu.kvbh, pol_kv);
+          tma_load_3d(base + L::kVOff + c * (kBlockN * 128), &tmV, BAR(L::kKVFull), c * 64, bu.jk * kBlockN, bu.kvbh, pol_kv);
         }
-        for (int i = bu.i0; i <= bu.i1; ++i, ++q_iter) {
+        for (int it = 0; it < bu.n_it; ++it, ++q_iter) {
+          const int i = bu.qtile(it), qbh = bu.qbh(it);
           const uint32_t st = q_iter % L::kStages, use = q_iter / L::kStages;
           if (use > 0 && !mbar_wait(BAR(L::kQEmpty + st), (use - 1) & 1, wc)) { ok = false; break; }
           const uint32_t fb = BAR(L::kQFull + st);
           mbar_arrive_expect_tx(fb, 2 * L::kQT + L::kVecStage);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) {
-            tma_load_3d(base + L::kQOff + st * L::kQT + c * (BR * 128), &tmQ, fb, c * 64, i * BR, bu.bh, pol_q);
-            tma_load_3d(base + L::kDOOff + st * L::kQT + c * (BR * 128), &tmDO, fb, c * 64, i * BR, bu.bh, pol_q);
+            tma_load_3d(base + L::kQOff + st * L::kQT + c * (BR * 128), &tmQ, fb, c * 64, i * BR, qbh, pol_q);
+            tma_load_3d(base + L::kDOOff + st * L::kQT + c * (BR * 128), &tmDO, fb, c * 64, i * BR, qbh, pol_q);
           }
-          const size_t row0 = (size_t)bu.bh * p.n_pad + (size_t)i * BR;
+          const size_t row0 = (size_t)qbh * p.n_pad + (size_t)i * BR;
           bulk_load(base + L::kVecOff + st * L::kVecStage, p.lse2 + row0, BR * 4, fb);
           bulk_load(base + L::kVecOff + st * L::kVecStage + BR * 4, p.dvec + row0, BR * 4, fb);
         }
@@ -247,11 +262,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mma_ss(tmem + L::kColS, kmaj<kBlockN>(sK, ks), kmaj<BR>(sQ, ks), idesc_s, ks > 0);
           tc_commit(BAR(L::kSFull));
         }
-        for (int i = bu.i0; i <= bu.i1; ++i, ++q_iter) {
+        for (int it = 0; it < bu.n_it; ++it, ++q_iter) {
           const uint32_t st = q_iter % L::kStages;
           const uint32_t sQ = base + L::kQOff + st * L::kQT;
           const uint32_t sDO = base + L::kDOOff + st * L::kQT;
-          const uint32_t first = (i == bu.i0);
+          const uint32_t first = (it == 0);
           // dP^T = V_j dO_i^T   (the dP region's previous contents, dS^T of
           // tile i-1, were consumed by dK(i-1), issued earlier)
 #pragma unroll
@@ -267,7 +282,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int ks = 0; ks < BR / 16; ++ks)
             mma_ts(tmem + L::kColDV, tmem + L::kColS + 8u * ks, mnmaj<BR>(sDO, ks), idesc_acc, (!first || ks > 0) ? 1u : 0u);
           // S^T for the next query tile (the S region's P^T was consumed by dV above)
-          if (i < bu.i1) {
+          if (it + 1 < bu.n_it) {
             const uint32_t st1 = (q_iter + 1) % L::kStages;
             if (!mbar_wait(BAR(L::kQFull + st1), ((q_iter + 1) / L::kStages) & 1, wc)) { ok = false; break; }
             tc_fence_after();
@@ -320,7 +335,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
       const int key = bu.jk * kBlockN + key_in;
       const bool key_ok = key < p.N;
-      for (int i = bu.i0; i <= bu.i1; ++i, ++q_iter) {
+      for (int it = 0; it < bu.n_it; ++it, ++q_iter) {
+        const int i = bu.qtile(it);
         const uint32_t st = q_iter % L::kStages;
         ok = warp_all(mbar_wait(BAR(L::kQFull + st), (q_iter / L::kStages) & 1, wc));
         if (!ok) break;
@@ -417,7 +433,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
       const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
-      for (int i = bu.i0; i <= bu.i1; ++i) {
+      for (int it = 0; it < bu.n_it; ++it) {
+        const int i = bu.qtile(it), qbh = bu.qbh(it);
         ok = warp_all(mbar_wait(BAR(L::kDQFull), dq_cnt & 1, wc));
         if (!ok) break;
         ++dq_cnt;
@@ -480,7 +497,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         fence_async_smem();
         named_bar_sync(1, 128);
         if (t == 0) {
-          bulk_reduce_add_f32(p.dq_acc + ((size_t)bu.bh * p.n_pad + (size_t)i * BR) * D, stage_s, L::kStage);
+          bulk_reduce_add_f32(p.dq_acc + ((size_t)qbh * p.n_pad + (size_t)i * BR) * D, stage_s, L::kStage);
           bulk_commit();
         }
       }
@@ -491,7 +508,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const int key = bu.jk * kBlockN + t;
       const bool in_range = key < p.N;
-      const size_t rowoff = ((size_t)bu.bh * p.N + (size_t)(in_range ? key : 0)) * D * 2;
+      const size_t rowoff = ((size_t)bu.kvbh * p.N + (size_t)(in_range ? key : 0)) * D * 2;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t col = which ? L::kColDK : L::kColDV;

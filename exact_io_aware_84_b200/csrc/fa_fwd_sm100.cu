@@ -64,15 +64,19 @@ template <int D>
 struct FwdLayout {
   static constexpr int kTile = kBlockM * D * 2;  // bytes of one 128 x D 16-bit tile
   static constexpr int kSlots = (D == 128) ? FA_FWD_SLOTS_D128 : 8;  // K/V ring depth (tiles)
+  // Q buffers (each holds the unit's two query tiles).  A second buffer, to
+  // prefetch the next unit's Q, measured no faster at d = 64 (the unit
+  // boundary is dominated by the causal tile imbalance), so one is used.
+  static constexpr int kQBufs = 1;
   static constexpr int kQOff = 0;
-  static constexpr int kKVOff = 2 * kTile;
+  static constexpr int kKVOff = kQBufs * 2 * kTile;
   static constexpr int kBarOff = kKVOff + kSlots * kTile;
   // barrier indices
-  static constexpr int kQFull = 0;
-  static constexpr int kQEmpty = 1;
-  static constexpr int kKVFull = 2;
-  static constexpr int kKVEmpty = 2 + kSlots;
-  static constexpr int kSFull = 2 + 2 * kSlots;  // [2]
+  static constexpr int kQFull = 0;                  // [kQBufs]
+  static constexpr int kQEmpty = kQBufs;            // [kQBufs]
+  static constexpr int kKVFull = 2 * kQBufs;
+  static constexpr int kKVEmpty = kKVFull + kSlots;
+  static constexpr int kSFull = kKVEmpty + kSlots;  // [2]
   static constexpr int kPFull = kSFull + 2;      // [2]
   static constexpr int kOFull = kPFull + 2;      // [2]
   static constexpr int kOEmpty = kOFull + 2;     // [2]
@@ -88,7 +92,8 @@ struct FwdLayout {
 };
 
 struct UnitInfo {
-  int bh;
+  int bh;    // batch * H + query head
+  int kvbh;  // batch * Hkv + key/value head read by that query head
   int r0_0, r0_1;  // first row of query tile 0 / 1
   int nb_0, nb_1;  // key/value tiles each query tile visits (0 = tile absent)
   int nmax;
@@ -107,6 +112,7 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams& p) {
     pair = u % p.n_pairs;
     ui.bh = u / p.n_pairs;
   }
+  ui.kvbh = (ui.bh / p.H) * (p.H / p.group) + (ui.bh % p.H) / p.group;
   ui.r0_0 = pair * 2 * kBlockM;
   ui.r0_1 = ui.r0_0 + kBlockM;
   ui.nb_0 = CAUSAL ? (ui.r0_0 / kBlockN + 1) : p.n_kv;  // tile 0 always exists
@@ -147,8 +153,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::kMiscOff + 4);
 
   if (threadIdx.x == 0) {
-    mbar_init(BAR(L::kQFull), 1);
-    mbar_init(BAR(L::kQEmpty), 1);
+    for (int b = 0; b < L::kQBufs; ++b) {
+      mbar_init(BAR(L::kQFull + b), 1);
+      mbar_init(BAR(L::kQEmpty + b), 1);
+    }
     for (int s = 0; s < L::kSlots; ++s) {
       mbar_init(BAR(L::kKVFull + s), 1);
       mbar_init(BAR(L::kKVEmpty + s), 1);
@@ -186,15 +194,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
         const UnitInfo ui = decode_unit<CAUSAL>(u, p);
-        if (unit_iter > 0 && !mbar_wait(BAR(L::kQEmpty), (unit_iter - 1) & 1, wc)) { ok = false; break; }
+        const uint32_t qb = unit_iter % L::kQBufs, quse = unit_iter / L::kQBufs;
+        if (quse > 0 && !mbar_wait(BAR(L::kQEmpty + qb), (quse - 1) & 1, wc)) { ok = false; break; }
         const uint32_t qbytes = (ui.nb_1 > 0 ? 2u : 1u) * L::kTile;
-        mbar_arrive_expect_tx(BAR(L::kQFull), qbytes);
+        mbar_arrive_expect_tx(BAR(L::kQFull + qb), qbytes);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           if (ui.nb(t) == 0) continue;
 #pragma unroll
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(base + L::kQOff + t * L::kTile + c * (kBlockM * 128), &tmQ, BAR(L::kQFull), c * 64,
+            tma_load_3d(base + L::kQOff + (qb * 2 + t) * L::kTile + c * (kBlockM * 128), &tmQ, BAR(L::kQFull + qb), c * 64,
                         ui.r0(t), ui.bh, pol_q);
         }
         for (int j = 0; j < ui.nmax && ok; ++j) {
@@ -205,7 +214,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_arrive_expect_tx(BAR(L::kKVFull + slot), L::kTile);
             for (int c = 0; c < D / 64; ++c)
               tma_load_3d(base + L::kKVOff + slot * L::kTile + c * (kBlockN * 128), kv ? &tmV : &tmK,
-                          BAR(L::kKVFull + slot), c * 64, j * kBlockN, ui.bh, pol_kv);
+                          BAR(L::kKVFull + slot), c * 64, j * kBlockN, ui.kvbh, pol_kv);
           }
         }
       }
@@ -215,7 +224,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const uint32_t issued = kv_iter / L::kSlots + (s < kv_iter % L::kSlots ? 1u : 0u);
           if (issued > 0) mbar_wait_drain(BAR(L::kKVFull + s), (issued - 1) & 1, p.wait_limit_ns);
         }
-        if (unit_iter > 0) mbar_wait_drain(BAR(L::kQFull), (unit_iter - 1) & 1, p.wait_limit_ns);
+        // unit_iter Q loads were issued (the aborted unit's included or not,
+        // both cases leave unit_iter equal to the number issued)
+        for (uint32_t b = 0; b < (uint32_t)L::kQBufs; ++b) {
+          const uint32_t issued = unit_iter / L::kQBufs + (b < unit_iter % L::kQBufs ? 1u : 0u);
+          if (issued > 0) mbar_wait_drain(BAR(L::kQFull + b), (issued - 1) & 1, p.wait_limit_ns);
+        }
       }
     }
   } else if (warp == kMmaWarp) {
@@ -228,7 +242,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
         const UnitInfo ui = decode_unit<CAUSAL>(u, p);
-        if (!mbar_wait(BAR(L::kQFull), unit_iter & 1, wc)) { ok = false; break; }
+        const uint32_t qb = unit_iter % L::kQBufs;
+        if (!mbar_wait(BAR(L::kQFull + qb), (unit_iter / L::kQBufs) & 1, wc)) { ok = false; break; }
         tc_fence_after();
         const uint32_t kv_base = kv_iter;
         for (int j = 0; j <= ui.nmax && ok; ++j) {
@@ -269,7 +284,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 tc_fence_after();
               }
               // S_t = Q_t K_j^T
-              const uint32_t qt = base + L::kQOff + t * L::kTile;
+              const uint32_t qt = base + L::kQOff + (qb * 2 + t) * L::kTile;
               const uint32_t kt = base + L::kKVOff + (k_idx % L::kSlots) * L::kTile;
 #pragma unroll
               for (int ks = 0; ks < D / 16; ++ks)
@@ -278,7 +293,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
           }
           if (!ok) break;
-          if (j == ui.nmax - 1) tc_commit(BAR(L::kQEmpty));
+          if (j == ui.nmax - 1) tc_commit(BAR(L::kQEmpty + qb));
           // Release K_j as soon as the S MMAs of block j are issued (they are
           // its last readers) and V_{j-1} after the PV MMAs of block j-1; the
           // producer can then refill the slots about one block ahead.

@@ -15,7 +15,9 @@ struct FwdParams {
   void* o;             // [B*H, N, D] 16-bit, or fp32 when the O32 variant runs
   float* lse;          // [B*H, N] fp32
   int N;               // sequence length
-  int bh;              // B*H
+  int bh;              // B*H (query heads)
+  int H;               // query heads per batch entry
+  int group;           // query heads per key/value head (H / Hkv)
   int n_kv;            // ceil(N / 128): key/value tiles per head
   int n_pairs;         // ceil(N / 256): pairs of 128-row Q tiles per head
   int n_units;         // bh * n_pairs
@@ -27,6 +29,7 @@ struct FwdParams {
 
 struct BwdParams {
   const void* o;       // forward output, [B*H, N, D] (16-bit, or fp32 for O32)
+  // q, o, dout, dq are [B*H, N, D]; k, v, dk, dv are [B*Hkv, N, D]
   const void* dout;    // dO, [B*H, N, D]
   const float* lse;    // [B*H, N]
   void* dq;            // [B*H, N, D]
@@ -37,9 +40,10 @@ struct BwdParams {
   float* lse2;         // [B*H, n_pad] fp32 workspace (LSE_i * log2 e; +inf on padding)
   int N;
   int n_pad;           // ceil(N / 128) * 128
-  int bh;
+  int bh;              // B*H (query heads)
+  int group;           // query heads per key/value head (H / Hkv)
   int n_kv;            // ceil(N / 128)
-  int n_units;         // bh * n_kv
+  int n_units;         // B * Hkv * n_kv
   float scale;         // softmax scale
   float scale_log2;    // scale * log2(e)
   uint64_t wait_limit_ns;

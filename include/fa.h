@@ -141,6 +141,27 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
                    int causal, int dtype, void* stream);
 
+/*
+ * Grouped-query attention (GQA / MQA): H query heads share Hkv key/value
+ * heads; query head h reads key/value head h / (H / Hkv).  H must be a
+ * multiple of Hkv (Hkv = 1: multi-query; Hkv = H: same as fa_fwd / fa_bwd).
+ *   q, o, lse, dout, dq : [B, H, N, d] (lse [B, H, N]), as in fa_fwd / fa_bwd.
+ *   k, v, dk, dv        : [B, Hkv, N, d]; dk, dv are the gradients summed over
+ *                         the query heads of each group.
+ *   workspace           : fa_bwd_workspace_size(B, H, N, d) bytes (per query head).
+ * Everything else as fa_fwd / fa_bwd; Hkv <= 0 or H % Hkv != 0 returns
+ * FA_ERR_INVALID_ARG.  The backward keeps each key/value head's dK and dV in
+ * tensor memory while it walks every query head of its group.  Source:
+ * delect.ru glossary "FlashAttention", "What is confirmed" (the attention
+ * computation does not change the number of key/value heads, so grouping is
+ * independent of it).
+ */
+int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
+               int d, float scale, int causal, int dtype, void* stream);
+int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+               void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int N,
+               int d, float scale, int causal, int dtype, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fa_status_string(int status);
 

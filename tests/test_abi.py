@@ -118,3 +118,12 @@ def test_python_binding_rejects_cpu_tensors():
     q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         fa.fa_fwd(q, q, q)
+
+
+def test_gqa_argument_errors(lib):
+    p = 0x1000
+    assert lib.fa_fwd_gqa(p, p, p, p, p, 1, 6, 4, 128, 64, 0.125, 0, 0, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_gqa(p, p, p, p, p, 1, 6, 0, 128, 64, 0.125, 0, 0, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_bwd_gqa(p, p, p, p, p, p, p, p, p, 0x10000, 1 << 30, 1, 8, 3, 128, 64, 0.125, 0, 0,
+                          None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_gqa(p, p, p, p, p, 1, 8, 2, 128, 96, 0.125, 0, 0, None) == fa.FA_ERR_UNSUPPORTED
