@@ -13,4 +13,6 @@ from .attention import (  # noqa: F401
     fa1_fwd_ref,
     gqa_fwd_ref,
     gqa_bwd_ref,
+    blocksparse_fwd_ref,
+    blocksparse_bwd_ref,
 )

@@ -40,6 +40,14 @@ What it computes (all in float64, on whatever arrays it is handed):
   (the per-query-head gradients summed over the group).  The delect.ru
   glossary ("What is confirmed") notes that the attention computation does
   not change the number of key/value heads: grouping is orthogonal to it.
+* ``blocksparse_fwd_ref`` / ``blocksparse_bwd_ref`` -- block-sparse attention:
+  a boolean mask over 128 x 128 (query block, key block) tiles; scores in
+  inactive tiles are excluded (-inf) on top of the causal mask.  It is an
+  approximation of full attention (ultralytics glossary, "Flash Attention and
+  related terms": the block-sparse variant skips empty tiles; delect.ru
+  glossary, "What is confirmed": it is described separately as an
+  approximation).  A row whose keys are all excluded has O = 0 and
+  LSE = -inf, and contributes no gradient.
 * ``fa1_fwd_ref`` -- the per-step-normalised loop of the marketmaker.cc
   section "The Flash Attention algorithm" (query blocks outer, key/value blocks
   inner, O normalised by the running sum after every block).
@@ -69,6 +77,8 @@ __all__ = [
     "fa1_fwd_ref",
     "gqa_fwd_ref",
     "gqa_bwd_ref",
+    "blocksparse_fwd_ref",
+    "blocksparse_bwd_ref",
 ]
 
 
@@ -304,3 +314,63 @@ def gqa_bwd_ref(q, k, v, do, scale, causal=False, row_chunk=1024):
     dq, dk, dv = attn_bwd_ref(q, _repeat_kv(k, g), _repeat_kv(v, g), do, scale, causal, row_chunk)
     n, d = dk.shape[-2:]
     return dq, dk.reshape(B, Hkv, g, n, d).sum(2), dv.reshape(B, Hkv, g, n, d).sum(2)
+
+
+def _element_mask(n, block_mask, block):
+    """Expand a [n_qb, n_kb] tile mask to an [n, n] element mask (True = kept)."""
+    bm = np.asarray(block_mask, dtype=bool)
+    idx = np.arange(n) // block
+    return bm[idx[:, None], idx[None, :]]
+
+
+def _masked_scores(q, k, scale, causal, keep):
+    s = float(scale) * (_f64(q) @ _f64(k).T)
+    if causal:
+        s = np.where(_causal_mask(np.arange(s.shape[0]), s.shape[1]), -np.inf, s)
+    return np.where(keep, s, -np.inf)
+
+
+def blocksparse_fwd_ref(q, k, v, scale, causal, block_mask, block=128):
+    """Block-sparse forward for [..., N, d] inputs.  ``block_mask`` is
+    [..., n_qb, n_kb] (leading dims broadcast against the heads)."""
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    lead = q.shape[:-2]
+    n, d = q.shape[-2:]
+    bm = np.broadcast_to(np.asarray(block_mask, dtype=bool), lead + np.asarray(block_mask).shape[-2:])
+    qf, kf, vf = (x.reshape((-1,) + x.shape[-2:]) for x in (q, k, v))
+    bmf = bm.reshape((-1,) + bm.shape[-2:])
+    o = np.empty((qf.shape[0], n, vf.shape[-1]))
+    lse = np.empty((qf.shape[0], n))
+    for h in range(qf.shape[0]):
+        s = _masked_scores(qf[h], kf[h], scale, causal, _element_mask(n, bmf[h], block))
+        lse[h], p = _two_pass(s)
+        o[h] = p @ vf[h]
+    return o.reshape(lead + (n, vf.shape[-1])), lse.reshape(lead + (n,))
+
+
+def blocksparse_bwd_ref(q, k, v, do, scale, causal, block_mask, block=128):
+    """Gradient of the block-sparse forward (excluded scores carry none)."""
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    do = _f64(do)
+    lead = q.shape[:-2]
+    n = q.shape[-2]
+    bm = np.broadcast_to(np.asarray(block_mask, dtype=bool), lead + np.asarray(block_mask).shape[-2:])
+    qf, kf, vf, dof = (x.reshape((-1,) + x.shape[-2:]) for x in (q, k, v, do))
+    bmf = bm.reshape((-1,) + bm.shape[-2:])
+    dq, dk, dv = np.zeros_like(qf), np.zeros_like(kf), np.zeros_like(vf)
+    for h in range(qf.shape[0]):
+        s = _masked_scores(qf[h], kf[h], scale, causal, _element_mask(n, bmf[h], block))
+        _, p = _two_pass(s)
+        o = p @ vf[h]
+        dv[h] = p.T @ dof[h]
+        dp = dof[h] @ vf[h].T
+        D = np.sum(dof[h] * o, axis=-1, keepdims=True)
+        ds = p * (dp - D)
+        dq[h] = float(scale) * (ds @ kf[h])
+        dk[h] = float(scale) * (ds.T @ qf[h])
+    shp = lambda x, ref: x.reshape(lead + ref.shape[-2:])
+    return shp(dq, q), shp(dk, k), shp(dv, v)

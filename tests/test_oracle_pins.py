@@ -23,6 +23,7 @@ import torch
 
 from oracle import (attn_bwd_ref, attn_fwd_ref, attn_fwd_rows_ref,
                     attn_probs_ref, attn_scores_ref, fa1_fwd_ref,
+                    blocksparse_bwd_ref, blocksparse_fwd_ref,
                     gqa_bwd_ref, gqa_fwd_ref, online_fwd_ref)
 from exact_io_aware_84_b200.metrics import score_matrix_bytes
 
@@ -398,3 +399,75 @@ def test_gqa_gradient_matches_finite_differences(causal):
             x[idx] = old
             num[idx] = (lp - lm) / (2 * h_step)
         np.testing.assert_allclose(ana, num, rtol=1e-5, atol=1e-7)
+
+
+# ------------------------------------------------------------ block sparsity
+
+def _brute_masked(q, k, v, scale, keep):
+    """Explicit loops over the kept (query, key) pairs; empty rows give O = 0
+    and LSE = -inf."""
+    n, dv = len(q), len(v[0])
+    o = np.zeros((n, dv))
+    lse = np.full(n, -np.inf)
+    for i in range(n):
+        s = [(j, scale * sum(float(q[i][c]) * float(k[j][c]) for c in range(len(q[0]))))
+             for j in range(len(k)) if keep[i][j]]
+        if not s:
+            continue
+        mx = max(x for _, x in s)
+        tot = sum(math.exp(x - mx) for _, x in s)
+        lse[i] = mx + math.log(tot)
+        for j, x in s:
+            o[i] += math.exp(x - mx) / tot * np.asarray(v[j], dtype=float)
+    return o, lse
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_blocksparse_forward_brute_force(causal):
+    # blocks of 2 over 7 rows (4 blocks, the last one ragged); query block 1
+    # sees no key block at all, so its rows are empty
+    r = _rng(50 + causal)
+    n = 7
+    q, k, v = (r.standard_normal((n, 3)) for _ in range(3))
+    bm = np.array([[1, 0, 1, 1], [0, 0, 0, 0], [1, 1, 0, 1], [0, 1, 1, 1]], dtype=bool)
+    keep = [[bool(bm[i // 2, j // 2]) and (not causal or j <= i) for j in range(n)] for i in range(n)]
+    o, lse = blocksparse_fwd_ref(q, k, v, 0.8, causal, bm, block=2)
+    ob, lb = _brute_masked(q, k, v, 0.8, keep)
+    np.testing.assert_allclose(o, ob, atol=1e-14)
+    np.testing.assert_array_equal(np.isneginf(lse), np.isneginf(lb))
+    fin = np.isfinite(lb)
+    np.testing.assert_allclose(lse[fin], lb[fin], atol=1e-14)
+    assert np.all(o[2:4] == 0) and np.all(np.isneginf(lse[2:4]))
+
+
+def test_blocksparse_dense_mask_is_full_attention():
+    r = _rng(52)
+    q, k, v, do = (r.standard_normal((2, 2, 9, 4)) for _ in range(4))
+    bm = np.ones((5, 5), dtype=bool)
+    for a, b in zip(blocksparse_fwd_ref(q, k, v, 0.5, True, bm, block=2), attn_fwd_ref(q, k, v, 0.5, True)):
+        np.testing.assert_allclose(a, b, atol=1e-15)
+    for a, b in zip(blocksparse_bwd_ref(q, k, v, do, 0.5, True, bm, block=2), attn_bwd_ref(q, k, v, do, 0.5, True)):
+        np.testing.assert_allclose(a, b, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_blocksparse_gradient_matches_finite_differences(causal):
+    r = _rng(53 + causal)
+    n, d = 6, 3
+    q, k, v, do = (r.standard_normal((n, d)) for _ in range(4))
+    bm = np.array([[1, 0, 1], [1, 1, 0], [0, 0, 0]], dtype=bool)  # last query block empty
+    keep = [[bool(bm[i // 2, j // 2]) and (not causal or j <= i) for j in range(n)] for i in range(n)]
+    scale, h = 0.7, 1e-6
+    dq, dk, dv = blocksparse_bwd_ref(q, k, v, do, scale, causal, bm, block=2)
+    for x, ana in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + h
+            lp = float(np.sum(do * _brute_masked(q, k, v, scale, keep)[0]))
+            x[idx] = old - h
+            lm = float(np.sum(do * _brute_masked(q, k, v, scale, keep)[0]))
+            x[idx] = old
+            num[idx] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(ana, num, rtol=1e-5, atol=1e-7)
+    assert np.all(dq[4:] == 0)  # empty rows: no gradient
