@@ -25,6 +25,8 @@ __all__ = [
     "fa_bwd_noalloc",
     "fa_fwd_gqa",
     "fa_bwd_gqa",
+    "fa_fwd_blocksparse",
+    "fa_bwd_blocksparse",
     "fa_status_string",
     "fa_last_device_status",
     "fa_debug_set_wait_limit_ms",
@@ -68,6 +70,10 @@ _SIGNATURES = {
                             _c_int, _vp]),
     "fa_bwd_gqa": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                             _c_int, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _vp]),
+    "fa_fwd_blocksparse": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_longlong, _c_int, _c_int, _c_int,
+                                    _c_int, _c_float, _c_int, _c_int, _vp]),
+    "fa_bwd_blocksparse": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_longlong, _vp, _vp, _vp, _vp,
+                                    _sz, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _vp]),
     "fa_bwd_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _vp]),
     "fa_status_string": (ctypes.c_char_p, [_c_int]),
@@ -344,4 +350,71 @@ def fa_bwd_gqa(q, k, v, o, do, lse, dq=None, dk=None, dv=None, workspace=None,
                                    _stream_handle(stream))
     if st != FA_OK:
         raise FAError(st, "fa_bwd_gqa")
+    return dq, dk, dv
+
+
+def _check_mask(block_mask, q):
+    torch = _torch()
+    B, H, N, _ = q.shape
+    nb = (N + 127) // 128
+    if not block_mask.is_cuda or block_mask.dtype != torch.uint8 or not block_mask.is_contiguous():
+        raise ValueError("block_mask must be a contiguous CUDA uint8 tensor")
+    if tuple(block_mask.shape[-2:]) != (nb, nb):
+        raise ValueError(f"block_mask must end in ({nb}, {nb}) for N = {N}")
+    if block_mask.dim() == 2:
+        return 0
+    if tuple(block_mask.shape) != (B, H, nb, nb):
+        raise ValueError("block_mask must be [nb, nb] (shared) or [B, H, nb, nb]")
+    return nb * nb
+
+
+def fa_fwd_blocksparse(q, k, v, block_mask, o=None, lse=None, scale: Optional[float] = None,
+                       causal: bool = False, stream=None, o_fp32: bool = False):
+    """Forward that skips the 128 x 128 tiles where ``block_mask`` (uint8,
+    [nb, nb] shared or [B, H, nb, nb], nb = ceil(N/128)) is 0."""
+    torch = _torch()
+    _check_bhnd("q", q)
+    _check_bhnd("k", k, q)
+    _check_bhnd("v", v, q)
+    stride = _check_mask(block_mask, q)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    if o is None:
+        o = torch.empty(q.shape, dtype=torch.float32 if o_fp32 else q.dtype, device=q.device)
+    else:
+        _check_bhnd("o", o, q, allow_f32=True)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    st = load_library().fa_fwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                           block_mask.data_ptr(), stride, B, H, N, d, float(scale),
+                                           int(bool(causal)), _dtype_code(q, o), _stream_handle(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd_blocksparse")
+    return o, lse
+
+
+def fa_bwd_blocksparse(q, k, v, o, do, lse, block_mask, dq=None, dk=None, dv=None, workspace=None,
+                       scale: Optional[float] = None, causal: bool = False, stream=None):
+    """Backward of fa_fwd_blocksparse (the same mask)."""
+    torch = _torch()
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _check_bhnd(name, t, None if name == "q" else q, allow_f32=(name == "o"))
+    stride = _check_mask(block_mask, q)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    need = fa_bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = load_library().fa_bwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                           lse.data_ptr(), block_mask.data_ptr(), stride, dq.data_ptr(),
+                                           dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                                           workspace.numel() * workspace.element_size(), B, H, N, d, float(scale),
+                                           int(bool(causal)), _dtype_code(q, o), _stream_handle(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd_blocksparse")
     return dq, dk, dv

@@ -156,8 +156,10 @@ int fa_debug_exp2_poly(const float* x, float* y, int n, void* stream) {
 }
 
 static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
-                    int N, int d, float scale, int causal, int dtype, void* stream) {
+                    int N, int d, float scale, int causal, int dtype, void* stream,
+                    const unsigned char* bmask = nullptr, long long bmask_stride = 0) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (bmask_stride < 0) return FA_ERR_INVALID_ARG;
   int st = check_common(B, H, N, d, scale, dtype);
   if (st != FA_OK) return st;
   if (Hkv <= 0 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
@@ -186,6 +188,8 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   p.scale_log2 = scale * kLog2e;
   p.wait_limit_ns = wait_limit_ns();
   p.debug_flags = g_debug_flags.load();
+  p.bmask = bmask;
+  p.bmask_stride = bmask_stride;
   if (!(p.status = status_ptr())) return FA_ERR_CUDA;
   const int grid = p.n_units < di.sms ? p.n_units : di.sms;
   cudaError_t e = launch_fwd(d, bf16, o32, causal != 0, tq, tk, tv, p, grid, static_cast<cudaStream_t>(stream));
@@ -212,8 +216,10 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
 
 static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
                     const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B,
-                    int H, int Hkv, int N, int d, float scale, int causal, int dtype, void* stream) {
+                    int H, int Hkv, int N, int d, float scale, int causal, int dtype, void* stream,
+                    const unsigned char* bmask = nullptr, long long bmask_stride = 0) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (bmask_stride < 0) return FA_ERR_INVALID_ARG;
   int st = check_common(B, H, N, d, scale, dtype);
   if (st != FA_OK) return st;
   if (Hkv <= 0 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
@@ -244,6 +250,8 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
   p.wait_limit_ns = wait_limit_ns();
+  p.bmask = bmask;
+  p.bmask_stride = bmask_stride;
   if (!(p.status = status_ptr())) return FA_ERR_CUDA;
   const size_t acc_bytes = ((size_t)bh * p.n_pad * d * sizeof(float) + 255) / 256 * 256;
   const size_t vec_bytes = ((size_t)bh * p.n_pad * sizeof(float) + 255) / 256 * 256;
@@ -274,6 +282,22 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const
                int d, float scale, int causal, int dtype, void* stream) {
   return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, N, d, scale, causal,
                   dtype, stream);
+}
+
+int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                       const unsigned char* block_mask, long long mask_head_stride, int B, int H, int N, int d,
+                       float scale, int causal, int dtype, void* stream) {
+  if (!block_mask) return FA_ERR_INVALID_ARG;
+  return fwd_impl(q, k, v, o, lse, B, H, H, N, d, scale, causal, dtype, stream, block_mask, mask_head_stride);
+}
+
+int fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                       const float* lse, const unsigned char* block_mask, long long mask_head_stride, void* dq,
+                       void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+                       float scale, int causal, int dtype, void* stream) {
+  if (!block_mask) return FA_ERR_INVALID_ARG;
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, H, N, d, scale, causal,
+                  dtype, stream, block_mask, mask_head_stride);
 }
 
 }  // extern "C"

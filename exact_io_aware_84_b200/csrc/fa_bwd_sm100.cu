@@ -68,7 +68,9 @@ struct BwdLayout {
   static constexpr int kSFull = kQEmpty + kStages, kDPFull = kSFull + 1, kPFull = kSFull + 2;
   static constexpr int kDSFull = kSFull + 3, kDSEmpty = kSFull + 4, kDQFull = kSFull + 5;
   static constexpr int kDQEmpty = kSFull + 6, kAccFull = kSFull + 7, kAccEmpty = kSFull + 8, kDrain = kSFull + 9;
-  static constexpr int kNumBars = kDrain + 1;
+  // dQ staging tile: free again (previous reduce has read it) / fully written
+  static constexpr int kStgFree = kSFull + 10, kStgDone = kSFull + 11;
+  static constexpr int kNumBars = kStgDone + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -79,6 +81,14 @@ struct BwdLayout {
   static constexpr uint32_t kColDK = 2 * BR + D;
   static constexpr uint32_t kColDQ = 2 * BR + 2 * D;
   static_assert(kColDQ + (D == 64 ? D : BR) <= 512, "tensor memory overflow");
+  // Compute warpgroup w (0, 1) owns query columns [w*HALF, (w+1)*HALF) of
+  // each tile and packs its 16-bit P^T / dS^T (two per 32-bit column) at the
+  // start of that range, so the two warpgroups never write columns the other
+  // still reads.  Column of the 16 queries of MMA K step ks:
+  static constexpr int HALF = BR / 2;
+  __host__ __device__ static constexpr uint32_t packed_col(int ks) {
+    return (uint32_t)((ks / (HALF / 16)) * HALF + (ks % (HALF / 16)) * 8);
+  }
   static_assert(kAlloc <= 232448, "shared memory overflow");
 };
 
@@ -116,6 +126,16 @@ __device__ __forceinline__ BUnit decode_bunit(int u, const BwdParams& p) {
   return r;
 }
 
+// Whether iteration `it` of the unit is computed: its query block attends the
+// unit's key block (always when dense).
+template <int D, bool SPARSE>
+__device__ __forceinline__ bool bactive(const BwdParams& p, const BUnit& bu, int it) {
+  if constexpr (!SPARSE) return true;
+  constexpr int BR = BwdLayout<D>::BR;
+  const int qblk = (bu.qtile(it) * BR) / kBlockN;
+  return p.bmask[(long long)bu.qbh(it) * p.bmask_stride + (long long)qblk * p.n_kv + bu.jk] != 0;
+}
+
 // Tile of R rows x D columns stored as D/64 column blocks of R x 128 B (SW128).
 // K-major operand view: advance 16 elements (32 B) per K step.
 template <int R>
@@ -144,7 +164,7 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, bool SPARSE>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_main(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -171,14 +191,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(BAR(L::kSFull), 1);
     mbar_init(BAR(L::kDPFull), 1);
-    mbar_init(BAR(L::kPFull), 128);
-    mbar_init(BAR(L::kDSFull), 128);
+    mbar_init(BAR(L::kPFull), 256);
+    mbar_init(BAR(L::kDSFull), 256);
     mbar_init(BAR(L::kDSEmpty), 1);
     mbar_init(BAR(L::kDQFull), 1);
-    mbar_init(BAR(L::kDQEmpty), 128);
+    mbar_init(BAR(L::kDQEmpty), 256);
     mbar_init(BAR(L::kAccFull), 1);
-    mbar_init(BAR(L::kAccEmpty), 128);
+    mbar_init(BAR(L::kAccEmpty), 256);
     mbar_init(BAR(L::kDrain), 1);
+    mbar_init(BAR(L::kStgFree), 1);
+    mbar_init(BAR(L::kStgDone), 256);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -214,7 +236,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tma_load_3d(base + L::kKOff + c * (kBlockN * 128), &tmK, BAR(L::kKVFull), c * 64, bu.jk * kBlockN, bu.kvbh, pol_kv);
           tma_load_3d(base + L::kVOff + c * (kBlockN * 128), &tmV, BAR(L::kKVFull), c * 64, bu.jk * kBlockN, bu.kvbh, pol_kv);
         }
-        for (int it = 0; it < bu.n_it; ++it, ++q_iter) {
+        for (int it = 0; it < bu.n_it; ++it) {
+          if (!bactive<D, SPARSE>(p, bu, it)) continue;
           const int i = bu.qtile(it), qbh = bu.qbh(it);
           const uint32_t st = q_iter % L::kStages, use = q_iter / L::kStages;
           if (use > 0 && !mbar_wait(BAR(L::kQEmpty + st), (use - 1) & 1, wc)) { ok = false; break; }
@@ -228,6 +251,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const size_t row0 = (size_t)qbh * p.n_pad + (size_t)i * BR;
           bulk_load(base + L::kVecOff + st * L::kVecStage, p.lse2 + row0, BR * 4, fb);
           bulk_load(base + L::kVecOff + st * L::kVecStage + BR * 4, p.dvec + row0, BR * 4, fb);
+          ++q_iter;
         }
       }
       if (!ok) {
@@ -251,8 +275,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
         if (!mbar_wait(BAR(L::kKVFull), unit_iter & 1, wc)) { ok = false; break; }
         const uint32_t sK = base + L::kKOff, sV = base + L::kVOff;
+        int a0 = 0;  // first computed iteration (n_it when the key tile is attended by none)
+        while (a0 < bu.n_it && !bactive<D, SPARSE>(p, bu, a0)) ++a0;
         // S^T for the first query tile
-        {
+        if (a0 < bu.n_it) {
           const uint32_t st = q_iter % L::kStages;
           if (!mbar_wait(BAR(L::kQFull + st), (q_iter / L::kStages) & 1, wc)) { ok = false; break; }
           tc_fence_after();
@@ -262,11 +288,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mma_ss(tmem + L::kColS, kmaj<kBlockN>(sK, ks), kmaj<BR>(sQ, ks), idesc_s, ks > 0);
           tc_commit(BAR(L::kSFull));
         }
-        for (int it = 0; it < bu.n_it; ++it, ++q_iter) {
+        for (int it = a0; it < bu.n_it; ++it) {
+          if (!bactive<D, SPARSE>(p, bu, it)) continue;
           const uint32_t st = q_iter % L::kStages;
           const uint32_t sQ = base + L::kQOff + st * L::kQT;
           const uint32_t sDO = base + L::kDOOff + st * L::kQT;
-          const uint32_t first = (it == 0);
+          const uint32_t first = (it == a0);
+          int nxt = it + 1;
+          while (nxt < bu.n_it && !bactive<D, SPARSE>(p, bu, nxt)) ++nxt;
           // dP^T = V_j dO_i^T   (the dP region's previous contents, dS^T of
           // tile i-1, were consumed by dK(i-1), issued earlier)
 #pragma unroll
@@ -280,9 +309,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < BR / 16; ++ks)
-            mma_ts(tmem + L::kColDV, tmem + L::kColS + 8u * ks, mnmaj<BR>(sDO, ks), idesc_acc, (!first || ks > 0) ? 1u : 0u);
+            mma_ts(tmem + L::kColDV, tmem + L::kColS + L::packed_col(ks), mnmaj<BR>(sDO, ks), idesc_acc, (!first || ks > 0) ? 1u : 0u);
           // S^T for the next query tile (the S region's P^T was consumed by dV above)
-          if (it + 1 < bu.n_it) {
+          if (nxt < bu.n_it) {
             const uint32_t st1 = (q_iter + 1) % L::kStages;
             if (!mbar_wait(BAR(L::kQFull + st1), ((q_iter + 1) / L::kStages) & 1, wc)) { ok = false; break; }
             tc_fence_after();
@@ -298,7 +327,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < BR / 16; ++ks)
-            mma_ts(tmem + L::kColDK, tmem + L::kColDP + 8u * ks, mnmaj<BR>(sQ, ks), idesc_acc, (!first || ks > 0) ? 1u : 0u);
+            mma_ts(tmem + L::kColDK, tmem + L::kColDP + L::packed_col(ks), mnmaj<BR>(sQ, ks), idesc_acc, (!first || ks > 0) ? 1u : 0u);
           // dQ_i (d=64) or dQ_i^T (d=128) from dS^T in shared memory
           if (dq_cnt > 0 && !mbar_wait(BAR(L::kDQEmpty), (dq_cnt - 1) & 1, wc)) { ok = false; break; }
           tc_fence_after();
@@ -314,6 +343,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           ++dq_cnt;
           tc_commit(BAR(L::kQEmpty + st));   // Q_i, dO_i, LSE_i, D_i no longer read
           tc_commit(BAR(L::kDSEmpty));       // dS^T shared tile no longer read
+          ++q_iter;
         }
         if (!ok) break;
         tc_commit(BAR(L::kAccFull));
@@ -322,37 +352,115 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_commit(BAR(L::kDrain));
       mbar_wait_drain(BAR(L::kDrain), 0, p.wait_limit_ns);
     }
-  } else if (warp < 4) {
-    // ---------------------------------------------------------------- softmax
-    const int key_in = threadIdx.x;  // 0..127 = TMEM lane
+  } else if (warp < 8) {
+    // ------------------------------------------------- compute warpgroups 0, 1
+    // Both warpgroups run the same loop on their own half of each query tile
+    // (queries [w*HALF, (w+1)*HALF)), thread = key = tensor-memory lane:
+    //   P^T half, arrive P; stage dQ of the previous iteration (half of its
+    //   columns), arrive dQ-empty; dS^T half, arrive dS.  At the end of a unit
+    //   each warpgroup writes half of the dims of dK and dV.
+    const int w = warp >> 2;                       // 0 or 1
+    const int key_in = threadIdx.x & 127;          // tensor-memory lane
+    const int tid256 = threadIdx.x;                // 0..255 over both warpgroups
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + L::kColS;
     const uint32_t tDP = tmem + lane_off + L::kColDP;
     const float sl2 = p.scale_log2;
-    uint32_t q_iter = 0, s_cnt = 0, dp_cnt = 0, ds_cnt = 0;
+    float* stage = reinterpret_cast<float*>(gbase + L::kStgOff);
+    const uint32_t stage_s = base + L::kStgOff;
+    constexpr int HALF = L::HALF;
+    constexpr int NC = HALF / 32;                  // 32-column chunks per warpgroup
+    uint32_t q_iter = 0, s_cnt = 0, dp_cnt = 0, ds_cnt = 0, dq_cnt = 0, unit_iter = 0;
+    int pend_qbh = -1, pend_i = 0;                 // dQ tile waiting to be staged
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+
+    // Stage the pending dQ tile: read this warpgroup's 32 columns of it from
+    // tensor memory (scaled), write them into the fp32 staging tile, then one
+    // thread adds the whole tile into the global accumulator.
+    auto stage_dq = [&]() -> bool {
+      // The two warpgroups meet on mbarriers with bounded waits, not on a
+      // named barrier: if one of them has given up on a timeout, the other
+      // must not wait for it forever.
+      const uint32_t sphase = dq_cnt & 1;
+      if (!warp_all(mbar_wait(BAR(L::kDQFull), sphase, wc))) return false;
+      ++dq_cnt;
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + L::kColDQ + 32u * w, v);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(BAR(L::kDQEmpty));
+      if (tid256 == 0) {
+        bulk_wait_read0();  // the previous reduce has finished reading the tile
+        mbar_arrive(BAR(L::kStgFree));
+      }
+      if (!warp_all(mbar_wait(BAR(L::kStgFree), sphase, wc))) return false;
+      if (D == 64) {
+        // lane = query key_in, columns = dims 32w..32w+31 of row key_in of the
+        // [128 queries][64 dims] tile; chunk positions rotated by key_in mod 8
+        // (static barrel shift of the registers) to spread banks.
+        const int rot = key_in & 7;
+#pragma unroll
+        for (int b = 1; b < 8; b <<= 1) {
+          if (rot & b) {
+            uint32_t tmp[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) tmp[e] = v[(e + 4 * b) & 31];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = tmp[e];
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int ch = 8 * w + ((e + key_in) & 7);
+          float4 f = make_float4(__uint_as_float(v[4 * e]) * p.scale, __uint_as_float(v[4 * e + 1]) * p.scale,
+                                 __uint_as_float(v[4 * e + 2]) * p.scale, __uint_as_float(v[4 * e + 3]) * p.scale);
+          *reinterpret_cast<float4*>(stage + key_in * 64 + 4 * ch) = f;
+        }
+      } else {
+        // lane = dim key_in, columns = queries 32w..32w+31: column key_in of
+        // the [64 queries][128 dims] tile
+#pragma unroll
+        for (int q = 0; q < 32; ++q) stage[(32 * w + q) * 128 + key_in] = __uint_as_float(v[q]) * p.scale;
+      }
+      fence_async_smem();
+      mbar_arrive(BAR(L::kStgDone));
+      bool good = true;
+      if (tid256 == 0) {
+        good = mbar_wait(BAR(L::kStgDone), sphase, wc);
+        if (good) {
+          bulk_reduce_add_f32(p.dq_acc + ((size_t)pend_qbh * p.n_pad + (size_t)pend_i * BR) * D, stage_s, L::kStage);
+          bulk_commit();
+        }
+      }
+      pend_qbh = -1;
+      return warp_all(good);
+    };
+
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
       const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
       const int key = bu.jk * kBlockN + key_in;
       const bool key_ok = key < p.N;
-      for (int it = 0; it < bu.n_it; ++it, ++q_iter) {
+      int n_done = 0;  // iterations computed in this unit
+      for (int it = 0; it < bu.n_it; ++it) {
+        if (!bactive<D, SPARSE>(p, bu, it)) continue;
         const int i = bu.qtile(it);
         const uint32_t st = q_iter % L::kStages;
         ok = warp_all(mbar_wait(BAR(L::kQFull + st), (q_iter / L::kStages) & 1, wc));
         if (!ok) break;
-        const float* lse2 = reinterpret_cast<const float*>(gbase + L::kVecOff + st * L::kVecStage);
+        const float* lse2 = reinterpret_cast<const float*>(gbase + L::kVecOff + st * L::kVecStage) + HALF * w;
         const float* dvec = lse2 + BR;
         ok = warp_all(mbar_wait(BAR(L::kSFull), s_cnt & 1, wc));
         if (!ok) break;
         ++s_cnt;
         tc_fence_after();
-        const int q0 = i * BR;
+        const int q0 = i * BR + HALF * w;  // first query of this warpgroup's half
         // P^T = exp2(S^T * scale*log2e - LSE*log2e), masked; kept packed
-        uint32_t pk[BR / 2];
+        uint32_t pk[HALF / 2];
 #pragma unroll
-        for (int c = 0; c < BR / 32; ++c) {
+        for (int c = 0; c < NC; ++c) {
           uint32_t r[32];
-          tmem_ld32(tS + 32u * c, r);
+          tmem_ld32(tS + HALF * w + 32u * c, r);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -364,11 +472,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             pk[16 * c + e] = pack2<BF16>(p0, p1);
           }
         }
+        // packed P^T of this half -> columns [HALF*w, HALF*w + HALF/2) of the
+        // S^T region, all of which this warpgroup has already read
 #pragma unroll
-        for (int c = 0; c < BR / 32; ++c) tmem_st16(tS + 16u * c, pk + 16 * c);
+        for (int c = 0; c < NC; ++c) tmem_st16(tS + HALF * w + 16u * c, pk + 16 * c);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(BAR(L::kPFull));
+        // dQ of the previous iteration (its MMA was issued after the previous
+        // dS; its tensor-memory tile is reused by this iteration's dQ MMA)
+        if (pend_qbh >= 0 && !(ok = stage_dq())) break;
         // dS^T = P^T o (dP^T - D)
         ok = warp_all(mbar_wait(BAR(L::kDPFull), dp_cnt & 1, wc));
         if (!ok) break;
@@ -377,15 +490,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = warp_all(ds_cnt == 0 || mbar_wait(BAR(L::kDSEmpty), (ds_cnt - 1) & 1, wc));
         if (!ok) break;
         ++ds_cnt;
-        // dS^T chunk by chunk (32 queries): into tensor memory for the dK MMA
-        // and into the SW128 shared tile [key][query] for the dQ MMA.  In
-        // the shared tile, column block cb holds queries 64cb..64cb+63 and
-        // 16-byte chunk ch of row `key_in` lives at position ch ^ (key_in & 7).
+        // dS^T chunk by chunk into tensor memory (for the dK MMA) and into the
+        // SW128 shared tile [key][query] (for the dQ MMA).  In the shared tile
+        // column block cb holds queries 64cb..64cb+63; 16-byte chunk ch of row
+        // key_in lives at position ch ^ (key_in & 7).  Packed dS^T chunk c goes
+        // to columns [HALF*w + 16c, +16): dP^T chunk c/2 of this half, read.
         uint8_t* ds_tile = gbase + L::kDSOff;
 #pragma unroll
-        for (int c = 0; c < BR / 32; ++c) {
+        for (int c = 0; c < NC; ++c) {
           uint32_t r[32];
-          tmem_ld32(tDP + 32u * c, r);
+          tmem_ld32(tDP + HALF * w + 32u * c, r);
           tmem_wait_ld();
           uint32_t dsk[16];
 #pragma unroll
@@ -405,14 +519,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const float ds1 = p1 * (__uint_as_float(r[2 * e + 1]) - dvec[qa + 1]);
             dsk[e] = pack2<BF16>(ds0, ds1);
           }
-          // dS^T chunk c goes to columns [16c, 16c+16) of the dP^T region:
-          // those belong to dP^T chunk c/2, already read; the chunks still to
-          // be read start at column 32(c+1) > 16c + 16.
-          tmem_st16(tDP + 16u * c, dsk);
-          const int cb = c >> 1;
+          tmem_st16(tDP + HALF * w + 16u * c, dsk);
+          const int qcol = HALF * w + 32 * c;  // first query of this chunk within the tile
+          const int cb = qcol >> 6;
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
-            const int ch = (c & 1) * 4 + h;
+            const int ch = ((qcol & 63) >> 3) + h;
             uint4 val = make_uint4(dsk[4 * h], dsk[4 * h + 1], dsk[4 * h + 2], dsk[4 * h + 3]);
             *reinterpret_cast<uint4*>(ds_tile + cb * (kBlockN * 128) + key_in * 128 + ((ch ^ (key_in & 7)) * 16)) = val;
           }
@@ -421,119 +533,49 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(L::kDSFull));
-      }
-    }
-  } else if (warp < 8) {
-    // ---------------------------------------------------------------- epilogue
-    const int t = threadIdx.x - 128;  // 0..127 = TMEM lane
-    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    float* stage = reinterpret_cast<float*>(gbase + L::kStgOff);
-    const uint32_t stage_s = base + L::kStgOff;
-    uint32_t dq_cnt = 0, unit_iter = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
-      const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
-      for (int it = 0; it < bu.n_it; ++it) {
-        const int i = bu.qtile(it), qbh = bu.qbh(it);
-        ok = warp_all(mbar_wait(BAR(L::kDQFull), dq_cnt & 1, wc));
-        if (!ok) break;
-        ++dq_cnt;
-        tc_fence_after();
-        // 64 fp32 columns per lane: d=64 -> lane = query, cols = dims;
-        //                           d=128 -> lane = dim, cols = queries.
-        if (D == 64) {
-          // lane t = query t, 64 fp32 columns = dims, staged as row t of the
-          // [128 queries][64 dims] tile.  Each 32-column half is read,
-          // scaled and written with its eight 16-byte chunks rotated by t mod 8
-          // (positions (e + t) mod 8 at step e), so lanes spread over all
-          // banks; the rotation is a static barrel shift of the registers.
-          uint32_t v[32];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            tmem_ld32(tmem + lane_off + L::kColDQ + 32u * h, v);
-            tmem_wait_ld();
-            if (h == 1) {
-              tc_fence_before();
-              mbar_arrive(BAR(L::kDQEmpty));
-            }
-            if (h == 0) {
-              // the previous bulk reduce must have finished reading the tile
-              if (t == 0) bulk_wait_read0();
-              named_bar_sync(1, 128);
-            }
-            const int rot = t & 7;
-#pragma unroll
-            for (int b = 1; b < 8; b <<= 1) {
-              if (rot & b) {
-                uint32_t tmp[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) tmp[e] = v[(e + 4 * b) & 31];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = tmp[e];
-              }
-            }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int ch = 8 * h + ((e + t) & 7);
-              float4 f = make_float4(__uint_as_float(v[4 * e]) * p.scale, __uint_as_float(v[4 * e + 1]) * p.scale,
-                                     __uint_as_float(v[4 * e + 2]) * p.scale, __uint_as_float(v[4 * e + 3]) * p.scale);
-              *reinterpret_cast<float4*>(stage + t * 64 + 4 * ch) = f;
-            }
-          }
-        } else {
-          // lane t = dim t, 64 fp32 columns = queries: column t of the
-          // [64 queries][128 dims] tile (consecutive lanes, consecutive words)
-          uint32_t v[64];
-          tmem_ld32(tmem + lane_off + L::kColDQ, v);
-          tmem_ld32(tmem + lane_off + L::kColDQ + 32, v + 32);
-          tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(BAR(L::kDQEmpty));
-          if (t == 0) bulk_wait_read0();
-          named_bar_sync(1, 128);
-#pragma unroll
-          for (int q = 0; q < 64; ++q) stage[q * 128 + t] = __uint_as_float(v[q]) * p.scale;
-        }
-        fence_async_smem();
-        named_bar_sync(1, 128);
-        if (t == 0) {
-          bulk_reduce_add_f32(p.dq_acc + ((size_t)qbh * p.n_pad + (size_t)i * BR) * D, stage_s, L::kStage);
-          bulk_commit();
-        }
+        pend_qbh = bu.qbh(it);
+        pend_i = i;
+        ++q_iter;
+        ++n_done;
       }
       if (!ok) break;
-      // dK, dV of this key tile: lane = key
+      // dK, dV of this key tile: lane = key, this warpgroup's half of the dims
       ok = warp_all(mbar_wait(BAR(L::kAccFull), unit_iter & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      const int key = bu.jk * kBlockN + t;
       const bool in_range = key < p.N;
       const size_t rowoff = ((size_t)bu.kvbh * p.N + (size_t)(in_range ? key : 0)) * D * 2;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
-        const uint32_t col = which ? L::kColDK : L::kColDV;
+        const uint32_t col = (which ? L::kColDK : L::kColDV) + (uint32_t)(D / 2) * w;
         const float mul = which ? p.scale : 1.f;
-        uint8_t* dst = reinterpret_cast<uint8_t*>(which ? p.dk : p.dv) + rowoff;
+        uint8_t* dst = reinterpret_cast<uint8_t*>(which ? p.dk : p.dv) + rowoff + (D / 2) * 2 * w;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t r[32];
-          tmem_ld32(tmem + lane_off + col + 32u * c, r);
-          tmem_wait_ld();
-          uint32_t w[16];
+          if (n_done > 0) {
+            tmem_ld32(tmem + lane_off + col + 32u * c, r);
+            tmem_wait_ld();
+          } else {  // no query attends this key tile: zero gradient
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = 0u;
+          }
+          uint32_t wv[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            w[e] = pack2<BF16>(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
+            wv[e] = pack2<BF16>(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
           if (in_range) {
             uint4* o = reinterpret_cast<uint4*>(dst + c * 64);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) o[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+            for (int e = 0; e < 4; ++e) o[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
           }
         }
       }
       tc_fence_before();
       mbar_arrive(BAR(L::kAccEmpty));
     }
-    if (t == 0) bulk_wait0();  // every dQ reduce has landed before the CTA exits
+    if (ok && pend_qbh >= 0) stage_dq();  // the CTA's last dQ tile
+    if (tid256 == 0) bulk_wait0();        // every dQ reduce has landed before the CTA exits
   }
 
   __syncwarp();
@@ -601,7 +643,10 @@ __global__ void __launch_bounds__(256) fa_bwd_prep(const BwdParams p) {
   const size_t prow = (size_t)bh * p.n_pad + row;
   if (lane == 0) {
     p.dvec[prow] = acc;
-    p.lse2[prow] = row < p.N ? p.lse[(size_t)bh * p.N + row] * 1.4426950408889634f : INFINITY;
+    // padding rows and rows with no kept key (LSE = -inf, block-sparse) get
+    // +inf, so that any P recomputed for them is 0
+    const float l = row < p.N ? p.lse[(size_t)bh * p.N + row] : -INFINITY;
+    p.lse2[prow] = l > -INFINITY ? l * 1.4426950408889634f : INFINITY;
   }
   float4* acc_row = reinterpret_cast<float4*>(p.dq_acc + prow * D);
 #pragma unroll
@@ -637,7 +682,7 @@ cudaError_t launch_bwd_t(bool o32, const CUtensorMap& tq, const CUtensorMap& tk,
     if (e != cudaSuccess) return e;
   }
   {
-    auto kern = fa_bwd_main<D, BF16, CAUSAL>;
+    auto kern = p.bmask ? fa_bwd_main<D, BF16, CAUSAL, true> : fa_bwd_main<D, BF16, CAUSAL, false>;
     constexpr int smem = BwdLayout<D>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;

@@ -95,13 +95,33 @@ struct UnitInfo {
   int bh;    // batch * H + query head
   int kvbh;  // batch * Hkv + key/value head read by that query head
   int r0_0, r0_1;  // first row of query tile 0 / 1
-  int nb_0, nb_1;  // key/value tiles each query tile visits (0 = tile absent)
+  int nb_0, nb_1;  // key/value tiles each query tile may visit (0 = tile absent)
   int nmax;
+  // Key/value tiles actually visited: the union of the two query tiles'
+  // active tiles (all of them when dense); each query tile visits those with
+  // index below its own nb, nbk_t of them.
+  int K, nbk_0, nbk_1;
   __device__ __forceinline__ int r0(int t) const { return t ? r0_1 : r0_0; }
   __device__ __forceinline__ int nb(int t) const { return t ? nb_1 : nb_0; }
+  __device__ __forceinline__ int nbk(int t) const { return t ? nbk_1 : nbk_0; }
 };
 
-template <bool CAUSAL>
+// Whether query block qblk of head bh attends key block kblk (dense: always).
+template <bool SPARSE>
+__device__ __forceinline__ bool tile_active(const FwdParams& p, int bh, int qblk, int kblk) {
+  if constexpr (!SPARSE) return true;
+  return p.bmask[(long long)bh * p.bmask_stride + (long long)qblk * p.n_kv + kblk] != 0;
+}
+// Key block j is visited by the unit when either query tile attends it.
+template <bool SPARSE>
+__device__ __forceinline__ bool unit_block(const FwdParams& p, const UnitInfo& ui, int j) {
+  if constexpr (!SPARSE) return j < ui.nmax;
+  const bool a0 = j < ui.nb_0 && tile_active<SPARSE>(p, ui.bh, ui.r0_0 / kBlockM, j);
+  const bool a1 = j < ui.nb_1 && tile_active<SPARSE>(p, ui.bh, ui.r0_1 / kBlockM, j);
+  return a0 || a1;
+}
+
+template <bool CAUSAL, bool SPARSE>
 __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams& p) {
   UnitInfo ui;
   int pair;
@@ -118,6 +138,18 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams& p) {
   ui.nb_0 = CAUSAL ? (ui.r0_0 / kBlockN + 1) : p.n_kv;  // tile 0 always exists
   ui.nb_1 = ui.r0_1 < p.N ? (CAUSAL ? (ui.r0_1 / kBlockN + 1) : p.n_kv) : 0;
   ui.nmax = ui.nb_1 > ui.nb_0 ? ui.nb_1 : ui.nb_0;
+  ui.K = ui.nmax;
+  ui.nbk_0 = ui.nb_0;
+  ui.nbk_1 = ui.nb_1;
+  if constexpr (SPARSE) {
+    ui.K = ui.nbk_0 = ui.nbk_1 = 0;
+    for (int j = 0; j < ui.nmax; ++j) {
+      if (!unit_block<SPARSE>(p, ui, j)) continue;
+      ++ui.K;
+      if (j < ui.nb_0) ++ui.nbk_0;
+      if (j < ui.nb_1) ++ui.nbk_1;
+    }
+  }
   return ui;
 }
 
@@ -136,7 +168,7 @@ __device__ __forceinline__ uint64_t v_desc(uint32_t tile, int kstep) {
   return make_sdesc_sw128(tile + (uint32_t)kstep * 2048, kBlockN * 128, 1024);
 }
 
-template <int D, bool BF16, bool O32, bool CAUSAL>
+template <int D, bool BF16, bool O32, bool CAUSAL, bool SPARSE>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -193,7 +225,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       uint32_t kv_iter = 0, unit_iter = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
-        const UnitInfo ui = decode_unit<CAUSAL>(u, p);
+        const UnitInfo ui = decode_unit<CAUSAL, SPARSE>(u, p);
         const uint32_t qb = unit_iter % L::kQBufs, quse = unit_iter / L::kQBufs;
         if (quse > 0 && !mbar_wait(BAR(L::kQEmpty + qb), (quse - 1) & 1, wc)) { ok = false; break; }
         const uint32_t qbytes = (ui.nb_1 > 0 ? 2u : 1u) * L::kTile;
@@ -207,6 +239,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         ui.r0(t), ui.bh, pol_q);
         }
         for (int j = 0; j < ui.nmax && ok; ++j) {
+          if (!unit_block<SPARSE>(p, ui, j)) continue;
           for (int kv = 0; kv < 2; ++kv, ++kv_iter) {
             const uint32_t slot = kv_iter % L::kSlots;
             const uint32_t use = kv_iter / L::kSlots;
@@ -241,17 +274,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       uint32_t p_cnt0 = 0, p_cnt1 = 0, o_uses0 = 0, o_uses1 = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
-        const UnitInfo ui = decode_unit<CAUSAL>(u, p);
+        const UnitInfo ui = decode_unit<CAUSAL, SPARSE>(u, p);
         const uint32_t qb = unit_iter % L::kQBufs;
         if (!mbar_wait(BAR(L::kQFull + qb), (unit_iter / L::kQBufs) & 1, wc)) { ok = false; break; }
         tc_fence_after();
         const uint32_t kv_base = kv_iter;
-        for (int j = 0; j <= ui.nmax && ok; ++j) {
+        if (ui.K == 0) tc_commit(BAR(L::kQEmpty + qb));  // no key block: Q is not read
+        for (int j = 0; j <= ui.K && ok; ++j) {          // j counts visited blocks
           const uint32_t k_idx = kv_base + 2 * j, v_idx = kv_base + 2 * (j - 1) + 1;
           bool v_ready = false, k_ready = false;
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
-            const int nbt = ui.nb(t);
+            const int nbt = ui.nbk(t);
             if (!ok || nbt == 0) continue;
             const uint32_t colS = L::kColS0 + 128u * t;
             const uint32_t colO = L::kColO0 + (uint32_t)D * t;
@@ -293,16 +327,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
           }
           if (!ok) break;
-          if (j == ui.nmax - 1) tc_commit(BAR(L::kQEmpty + qb));
+          if (j == ui.K - 1) tc_commit(BAR(L::kQEmpty + qb));
           // Release K_j as soon as the S MMAs of block j are issued (they are
           // its last readers) and V_{j-1} after the PV MMAs of block j-1; the
           // producer can then refill the slots about one block ahead.
-          if (j < ui.nmax) tc_commit(BAR(L::kKVEmpty + k_idx % L::kSlots));
+          if (j < ui.K) tc_commit(BAR(L::kKVEmpty + k_idx % L::kSlots));
           if (j >= 1) tc_commit(BAR(L::kKVEmpty + v_idx % L::kSlots));
         }
-        kv_iter = kv_base + 2 * ui.nmax;
-        o_uses0 += 1;
-        o_uses1 += ui.nb_1 > 0 ? 1u : 0u;
+        kv_iter = kv_base + 2 * ui.K;
+        o_uses0 += ui.nbk_0 > 0 ? 1u : 0u;
+        o_uses1 += ui.nbk_1 > 0 ? 1u : 0u;
       }
       // Make sure no MMA is still reading shared memory or writing tensor
       // memory when the CTA leaves (normal exit: they are all done already).
@@ -322,12 +356,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     int unit_iter = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
-      const UnitInfo ui = decode_unit<CAUSAL>(u, p);
-      const int nb = ui.nb(t);
-      if (nb == 0) continue;
+      const UnitInfo ui = decode_unit<CAUSAL, SPARSE>(u, p);
+      if (ui.nb(t) == 0) continue;                 // query tile past the sequence end
+      const int nb = ui.nbk(t);                    // key blocks this tile visits
       const int row = ui.r0(t) + r_in;
-      float m_run = -INFINITY, l_run = 0.f;
+      const int qblk = ui.r0(t) / kBlockM;
+      float m_run = -INFINITY, l_run = 0.f;        // m_run stays -inf until a key is seen
+      int jb = -1;                                 // index of the current key block
       for (int j = 0; j < nb; ++j) {
+        do { ++jb; } while (!unit_block<SPARSE>(p, ui, jb));
         ok = warp_all(mbar_wait(BAR(L::kSFull + t), s_cnt & 1, wc));
         if (!ok) break;
         ++s_cnt;
@@ -339,8 +376,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         float s[kBlockN];
 #pragma unroll
         for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(sr[c]);
-        const int kbase = j * kBlockN;
-        if (CAUSAL && j == nb - 1) {
+        const int kbase = jb * kBlockN;
+        if (SPARSE && !tile_active<SPARSE>(p, ui.bh, qblk, jb)) {
+          // visited for the other query tile only: nothing of it is kept here
+#pragma unroll
+          for (int c = 0; c < kBlockN; ++c) s[c] = -INFINITY;
+        } else if (CAUSAL && jb == qblk) {
 #pragma unroll
           for (int c = 0; c < kBlockN; ++c)
             if (kbase + c > row) s[c] = -INFINITY;
@@ -359,13 +400,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int a = 0; a < 8; ++a) pm[a] = fmax3(pm[a], s[c + a], s[c + a + 8]);
         const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
         const float m_new = fmaxf(m_run, mx * sl2);
-        if (j == 0) {
-          m_run = (m_new == -INFINITY) ? 0.f : m_new;
-        } else {
+        // Until a row has seen a key, its O and l are zero: the first finite
+        // max is taken as is, without a rescale.
+        const bool fresh = m_run == -INFINITY;
+        const bool need = !fresh && m_new > m_run + kRescaleThreshold;
+        if (fresh) m_run = m_new;
+        {
           // The rescale touches tensor memory with warp-collective
           // instructions, so the whole warp takes the branch when any of its
           // rows needs it; rows that do not keep their max and use alpha = 1.
-          const bool need = m_new > m_run + kRescaleThreshold;
           if (__any_sync(0xffffffffu, need)) {
             const float alpha = need ? ex2_approx(m_run - m_new) : 1.f;
             if (need) {
@@ -385,7 +428,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
           }
         }
-        const float neg_m = -m_run;
+        const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;  // -inf row: every P is 0
         float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int q = 0; q < kBlockN / 32; ++q) {
@@ -409,20 +452,29 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!withhold) mbar_arrive(BAR(L::kPFull + t));
       }
       if (!ok) break;
-      // ---- epilogue: O / l -> dtype -> global; LSE = (m + log2 l) ln 2
-      ok = warp_all(mbar_wait(BAR(L::kOFull + t), o_cnt & 1, wc));
-      if (!ok) break;
-      ++o_cnt;
-      tc_fence_after();
-      const float inv_l = 1.f / l_run;
+      // ---- epilogue: O / l -> dtype -> global; LSE = (m + log2 l) ln 2.
+      // A row with no kept key (block-sparse) gets O = 0 and LSE = -inf; a
+      // tile that visits no key block at all skips tensor memory entirely.
+      if (nb > 0) {
+        ok = warp_all(mbar_wait(BAR(L::kOFull + t), o_cnt & 1, wc));
+        if (!ok) break;
+        ++o_cnt;
+        tc_fence_after();
+      }
+      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
       const bool in_range = row < p.N;
       constexpr int kOBytes = O32 ? 4 : 2;
       uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + ((size_t)ui.bh * p.N + (size_t)(in_range ? row : 0)) * D * kOBytes;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(tO + 32u * c, o);
-        tmem_wait_ld();
+        if (nb > 0) {
+          tmem_ld32(tO + 32u * c, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
         if constexpr (O32) {
           if (in_range) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c * 128);
@@ -445,9 +497,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
         }
       }
-      tc_fence_before();
-      mbar_arrive(BAR(L::kOEmpty + t));
-      if (in_range) p.lse[(size_t)ui.bh * p.N + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+      if (nb > 0) {
+        tc_fence_before();
+        mbar_arrive(BAR(L::kOEmpty + t));
+      }
+      if (in_range)
+        p.lse[(size_t)ui.bh * p.N + row] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
     }
   }
 
@@ -460,10 +515,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 }
 
-template <int D, bool BF16, bool O32, bool CAUSAL>
+template <int D, bool BF16, bool O32, bool CAUSAL, bool SPARSE>
 cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const FwdParams& p, int grid, cudaStream_t st) {
-  auto kern = fa_fwd_kernel<D, BF16, O32, CAUSAL>;
+  auto kern = fa_fwd_kernel<D, BF16, O32, CAUSAL, SPARSE>;
   constexpr int smem = FwdLayout<D>::kAlloc;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -474,8 +529,11 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 template <int D, bool BF16, bool O32>
 cudaError_t launch_fwd_c(bool causal, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const FwdParams& p, int grid, cudaStream_t st) {
-  return causal ? launch_fwd_t<D, BF16, O32, true>(tq, tk, tv, p, grid, st)
-                : launch_fwd_t<D, BF16, O32, false>(tq, tk, tv, p, grid, st);
+  const bool sparse = p.bmask != nullptr;
+  if (causal) return sparse ? launch_fwd_t<D, BF16, O32, true, true>(tq, tk, tv, p, grid, st)
+                            : launch_fwd_t<D, BF16, O32, true, false>(tq, tk, tv, p, grid, st);
+  return sparse ? launch_fwd_t<D, BF16, O32, false, true>(tq, tk, tv, p, grid, st)
+                : launch_fwd_t<D, BF16, O32, false, false>(tq, tk, tv, p, grid, st);
 }
 
 template <int D>

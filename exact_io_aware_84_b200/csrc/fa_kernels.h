@@ -25,6 +25,10 @@ struct FwdParams {
   uint64_t wait_limit_ns;
   int* status;         // device status word
   int debug_flags;
+  // Block sparsity (nullptr = dense): uint8 [n_kv][n_kv] tile mask per query
+  // head, head h at bmask + h * bmask_stride (stride 0 = one mask for all).
+  const uint8_t* bmask;
+  long long bmask_stride;
 };
 
 struct BwdParams {
@@ -48,6 +52,8 @@ struct BwdParams {
   float scale_log2;    // scale * log2(e)
   uint64_t wait_limit_ns;
   int* status;         // device status word
+  const uint8_t* bmask;  // block sparsity as in FwdParams (nullptr = dense)
+  long long bmask_stride;
 };
 
 // Launchers (return cudaError_t of the launch).

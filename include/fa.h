@@ -162,6 +162,30 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const
                void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int N,
                int d, float scale, int causal, int dtype, void* stream);
 
+/*
+ * Block-sparse attention: whole 128 x 128 (query block, key block) tiles are
+ * skipped, never loaded nor computed, where the mask is 0 (on top of the
+ * causal mask when `causal` is set).  This approximates full attention; it
+ * equals it when every tile is kept.  Source: ultralytics.com glossary
+ * "Flash Attention", "Flash Attention and related terms" (the block-sparse
+ * variant skips empty tiles); delect.ru glossary "FlashAttention", "What is
+ * confirmed" (described separately as an approximation).
+ *   block_mask       : device uint8 [nb][nb] per query head, nb = ceil(N/128),
+ *                      row = query block, column = key block, non-zero = keep;
+ *                      head b*H + h starts at block_mask + (b*H + h) *
+ *                      mask_head_stride (0 = one mask for every head).
+ *   Other arguments as fa_fwd / fa_bwd.  A query row with no kept key gets
+ *   O = 0, LSE = -inf and zero gradients; a key with no query attending it
+ *   gets dK = dV = 0.  NULL mask or negative stride: FA_ERR_INVALID_ARG.
+ */
+int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                       const unsigned char* block_mask, long long mask_head_stride, int B, int H, int N, int d,
+                       float scale, int causal, int dtype, void* stream);
+int fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                       const float* lse, const unsigned char* block_mask, long long mask_head_stride, void* dq,
+                       void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+                       float scale, int causal, int dtype, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fa_status_string(int status);
 

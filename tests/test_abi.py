@@ -127,3 +127,12 @@ def test_gqa_argument_errors(lib):
     assert lib.fa_bwd_gqa(p, p, p, p, p, p, p, p, p, 0x10000, 1 << 30, 1, 8, 3, 128, 64, 0.125, 0, 0,
                           None) == fa.FA_ERR_INVALID_ARG
     assert lib.fa_fwd_gqa(p, p, p, p, p, 1, 8, 2, 128, 96, 0.125, 0, 0, None) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_blocksparse_rejects_null_mask_and_negative_stride():
+    lib = fa.load_library()
+    p = 0x1000
+    assert lib.fa_fwd_blocksparse(p, p, p, p, p, None, 0, 1, 1, 128, 64, 0.125, 0, 0, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_blocksparse(p, p, p, p, p, p, -1, 1, 1, 128, 64, 0.125, 0, 0, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_bwd_blocksparse(p, p, p, p, p, p, None, 0, p, p, p, p, 1 << 20, 1, 1, 128, 64, 0.125, 0, 0,
+                                  None) == fa.FA_ERR_INVALID_ARG
