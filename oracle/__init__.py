@@ -15,4 +15,8 @@ from .attention import (  # noqa: F401
     gqa_bwd_ref,
     blocksparse_fwd_ref,
     blocksparse_bwd_ref,
+    merge_partials_ref,
+    attn_bwd_partial_ref,
+    ring_fwd_ref,
+    ring_bwd_ref,
 )

@@ -48,6 +48,21 @@ What it computes (all in float64, on whatever arrays it is handed):
   glossary, "What is confirmed": it is described separately as an
   approximation).  A row whose keys are all excluded has O = 0 and
   LSE = -inf, and contributes no gradient.
+* ``merge_partials_ref`` / ``attn_bwd_partial_ref`` / ``ring_fwd_ref`` /
+  ``ring_bwd_ref`` -- ring attention: the sequence is split into equal chunks,
+  one per device; each device keeps its query chunk and computes attention
+  block by block against the key/value chunks as they pass around a ring
+  (ultralytics glossary, "Flash Attention and related terms", ring
+  attention).  A chunk's result is a partial (O, LSE) over that chunk's keys;
+  two partials over disjoint key sets combine as
+  LSE = ln(e^{LSE_a} + e^{LSE_b}), O = e^{LSE_a - LSE} O_a + e^{LSE_b - LSE} O_b,
+  which is the online-softmax recurrence of marketmaker.cc "Online softmax
+  recurrence" taken one whole chunk at a time.  With causal masking and chunks
+  aligned to the sequence, a key chunk before the query chunk is attended in
+  full, the same chunk with the causal mask, and a later chunk not at all.
+  The gradient of a chunk pair uses the full row statistics (the merged LSE
+  and O): P = exp(S - LSE), D = rowsum(dO o O), and the per-pair dQ, dK, dV
+  sum to the full gradient.
 * ``fa1_fwd_ref`` -- the per-step-normalised loop of the marketmaker.cc
   section "The Flash Attention algorithm" (query blocks outer, key/value blocks
   inner, O normalised by the running sum after every block).
@@ -78,6 +93,10 @@ __all__ = [
     "gqa_fwd_ref",
     "gqa_bwd_ref",
     "blocksparse_fwd_ref",
+    "merge_partials_ref",
+    "attn_bwd_partial_ref",
+    "ring_fwd_ref",
+    "ring_bwd_ref",
     "blocksparse_bwd_ref",
 ]
 
@@ -374,3 +393,102 @@ def blocksparse_bwd_ref(q, k, v, do, scale, causal, block_mask, block=128):
         dk[h] = float(scale) * (ds.T @ qf[h])
     shp = lambda x, ref: x.reshape(lead + ref.shape[-2:])
     return shp(dq, q), shp(dk, k), shp(dv, v)
+
+
+def merge_partials_ref(o_a, lse_a, o_b, lse_b):
+    """Combine two partial attention results of the same queries over
+    disjoint key sets.  o_*: [..., n, d]; lse_*: [..., n].  Rows where both
+    LSEs are -inf (no key seen yet) stay O = 0, LSE = -inf."""
+    o_a, lse_a, o_b, lse_b = (_f64(x) for x in (o_a, lse_a, o_b, lse_b))
+    m = np.maximum(lse_a, lse_b)
+    m_safe = np.where(np.isfinite(m), m, 0.0)
+    w_a = np.exp(lse_a - m_safe)      # e^{LSE_a - m}; 0 where LSE_a = -inf
+    w_b = np.exp(lse_b - m_safe)
+    tot = w_a + w_b
+    with np.errstate(divide="ignore"):
+        lse = np.where(tot > 0, m_safe + np.log(tot), -np.inf)
+    den = np.where(tot > 0, tot, 1.0)[..., None]
+    o = (w_a[..., None] * o_a + w_b[..., None] * o_b) / den
+    return o, lse
+
+
+def attn_bwd_partial_ref(q, k, v, o, do, lse, scale, causal=False):
+    """Gradient contributions of one key/value chunk to rows whose full
+    output O and log-sum-exp LSE are given (computed over all keys):
+    P = exp(S - LSE), dV = P^T dO, dP = dO V^T, D = rowsum(dO o O),
+    dS = P o (dP - D), dQ = scale dS K, dK = scale dS^T Q.  Inputs
+    [..., n, d] (q, o, do), [..., m, d] (k, v), [..., n] (lse)."""
+    q, k, v, o, do, lse = (_f64(x) for x in (q, k, v, o, do, lse))
+    lead = q.shape[:-2]
+    n, d = q.shape[-2:]
+    qf, of, dof = (x.reshape((-1, n, x.shape[-1])) for x in (q, o, do))
+    kf, vf = (x.reshape((-1,) + x.shape[-2:]) for x in (k, v))
+    lf = lse.reshape((-1, n))
+    dq, dk, dv = np.zeros_like(qf), np.zeros_like(kf), np.zeros_like(vf)
+    for h in range(qf.shape[0]):
+        s, _ = attn_scores_ref(qf[h], kf[h], scale, causal)
+        with np.errstate(invalid="ignore"):
+            p = np.where(np.isfinite(lf[h])[:, None], np.exp(s - lf[h][:, None]), 0.0)
+        dv[h] = p.T @ dof[h]
+        dp = dof[h] @ vf[h].T
+        D = np.sum(dof[h] * of[h], axis=-1, keepdims=True)
+        ds = p * (dp - D)
+        dq[h] = float(scale) * (ds @ kf[h])
+        dk[h] = float(scale) * (ds.T @ qf[h])
+    return dq.reshape(lead + (n, d)), dk.reshape(k.shape), dv.reshape(v.shape)
+
+
+def _ring_pairs(world, causal):
+    """(rank, step, source chunk, chunk-causal) in ring order: at step s rank
+    r holds the key/value chunk that started on rank (r - s) mod world."""
+    for r in range(world):
+        for step in range(world):
+            src = (r - step) % world
+            if causal and src > r:
+                continue            # every key of that chunk is in the future
+            yield r, step, src, causal and src == r
+
+
+def _chunks(x, world):
+    n = x.shape[-2]
+    if n % world:
+        raise ValueError("sequence length must be a multiple of the ring size")
+    c = n // world
+    return [x[..., i * c:(i + 1) * c, :] for i in range(world)]
+
+
+def ring_fwd_ref(q, k, v, scale, causal=False, world=2):
+    """Forward by the ring schedule: per rank, merge the partial results of
+    its query chunk against each key/value chunk in the order they arrive.
+    Inputs [..., N, d] with N a multiple of ``world``; returns (O, LSE)."""
+    q, k, v = (_f64(x) for x in (q, k, v))
+    qs, ks, vs = (_chunks(x, world) for x in (q, k, v))
+    o = [None] * world
+    lse = [None] * world
+    for r, _, src, diag in _ring_pairs(world, causal):
+        o_p, l_p = attn_fwd_ref(qs[r], ks[src], vs[src], scale, diag)
+        if o[r] is None:
+            o[r], lse[r] = o_p, l_p
+        else:
+            o[r], lse[r] = merge_partials_ref(o[r], lse[r], o_p, l_p)
+    return np.concatenate(o, axis=-2), np.concatenate(lse, axis=-1)
+
+
+def ring_bwd_ref(q, k, v, do, scale, causal=False, world=2):
+    """Gradient by the ring schedule: O and LSE from ``ring_fwd_ref``, then
+    per (rank, chunk) pair the partial gradients, dQ summed on the query's
+    rank and dK, dV summed for the chunk's owner."""
+    q, k, v, do = (_f64(x) for x in (q, k, v, do))
+    o, lse = ring_fwd_ref(q, k, v, scale, causal, world)
+    qs, ks, vs, os_, dos = (_chunks(x, world) for x in (q, k, v, o, do))
+    ls = [lse[..., i * (q.shape[-2] // world):(i + 1) * (q.shape[-2] // world)] for i in range(world)]
+    dq = [np.zeros_like(x) for x in qs]
+    dk = [np.zeros_like(x) for x in ks]
+    dv = [np.zeros_like(x) for x in vs]
+    for r, _, src, diag in _ring_pairs(world, causal):
+        gq, gk, gv = attn_bwd_partial_ref(qs[r], ks[src], vs[src], os_[r], dos[r], ls[r], scale, diag)
+        dq[r] += gq
+        dk[src] += gk
+        dv[src] += gv
+    cat = lambda xs: np.concatenate(xs, axis=-2)
+    return cat(dq), cat(dk), cat(dv)

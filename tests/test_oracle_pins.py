@@ -24,7 +24,9 @@ import torch
 from oracle import (attn_bwd_ref, attn_fwd_ref, attn_fwd_rows_ref,
                     attn_probs_ref, attn_scores_ref, fa1_fwd_ref,
                     blocksparse_bwd_ref, blocksparse_fwd_ref,
-                    gqa_bwd_ref, gqa_fwd_ref, online_fwd_ref)
+                    gqa_bwd_ref, gqa_fwd_ref, online_fwd_ref,
+                    attn_bwd_partial_ref, merge_partials_ref, ring_bwd_ref,
+                    ring_fwd_ref)
 from exact_io_aware_84_b200.metrics import score_matrix_bytes
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -471,3 +473,102 @@ def test_blocksparse_gradient_matches_finite_differences(causal):
             num[idx] = (lp - lm) / (2 * h)
         np.testing.assert_allclose(ana, num, rtol=1e-5, atol=1e-7)
     assert np.all(dq[4:] == 0)  # empty rows: no gradient
+
+
+
+# ---------------------------------------------------------------- ring attention
+
+def test_merge_of_disjoint_key_sets_is_brute_force_of_their_union():
+    r = _rng(61)
+    n, m, d = 5, 9, 3
+    q, k, v = r.standard_normal((n, d)), r.standard_normal((m, d)), r.standard_normal((m, d))
+    # interleaved, uneven split of the keys; row 4 sees keys of one set only
+    in_a = [[j % 3 == 0 for j in range(m)] for _ in range(n)]
+    in_b = [[j % 3 != 0 for j in range(m)] for _ in range(n)]
+    in_b[4] = [False] * m
+    both = [[a or b for a, b in zip(ra, rb)] for ra, rb in zip(in_a, in_b)]
+    oa, la = _brute_masked(q, k, v, 0.6, in_a)
+    ob, lb = _brute_masked(q, k, v, 0.6, in_b)
+    o, lse = merge_partials_ref(oa, la, ob, lb)
+    o_ref, l_ref = _brute_masked(q, k, v, 0.6, both)
+    np.testing.assert_allclose(o, o_ref, atol=1e-14)
+    np.testing.assert_allclose(lse, l_ref, atol=1e-14)
+
+
+def test_merge_special_cases():
+    r = _rng(62)
+    o1, l1 = r.standard_normal((4, 3)), r.standard_normal(4)
+    empty_o, empty_l = np.zeros((4, 3)), np.full(4, -np.inf)
+    for o, lse in (merge_partials_ref(o1, l1, empty_o, empty_l), merge_partials_ref(empty_o, empty_l, o1, l1)):
+        np.testing.assert_array_equal(o, o1)
+        np.testing.assert_array_equal(lse, l1)
+    o, lse = merge_partials_ref(empty_o, empty_l, empty_o, empty_l)
+    assert not o.any() and np.all(np.isneginf(lse))
+    # two copies of one partial: same O, LSE + ln 2
+    o, lse = merge_partials_ref(o1, l1, o1, l1)
+    np.testing.assert_allclose(o, o1, atol=1e-15)
+    np.testing.assert_allclose(lse, l1 + math.log(2.0), atol=1e-15)
+    # the heavier partial dominates: LSE_b = LSE_a + ln 3 gives weights 1/4, 3/4
+    o2 = r.standard_normal((4, 3))
+    o, lse = merge_partials_ref(o1, l1, o2, l1 + math.log(3.0))
+    np.testing.assert_allclose(o, 0.25 * o1 + 0.75 * o2, atol=1e-14)
+    np.testing.assert_allclose(lse, l1 + math.log(4.0), atol=1e-14)
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_forward_is_brute_force(world, causal):
+    r = _rng(63 + world)
+    n, d = 12, 3
+    q, k, v = (r.standard_normal((n, d)) for _ in range(3))
+    o, lse = ring_fwd_ref(q, k, v, 0.9, causal, world)
+    ob, lb = _brute_fwd(q.tolist(), k.tolist(), v.tolist(), 0.9, causal)
+    np.testing.assert_allclose(o, np.array(ob), atol=1e-14)
+    np.testing.assert_allclose(lse, np.array(lb), atol=1e-14)
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_gradient_matches_finite_differences(world, causal):
+    r = _rng(71 + world + 2 * causal)
+    n, d = 6, 2
+    q, k, v, do = (r.standard_normal((n, d)) for _ in range(4))
+    scale, h = 0.8, 1e-6
+    dq, dk, dv = ring_bwd_ref(q, k, v, do, scale, causal, world)
+    loss = lambda: sum(float(a) * float(b) for ra, rb in zip(do.tolist(), _brute_fwd(q.tolist(), k.tolist(), v.tolist(), scale, causal)[0]) for a, b in zip(ra, rb))
+    for x, ana in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + h
+            lp = loss()
+            x[idx] = old - h
+            lm = loss()
+            x[idx] = old
+            num[idx] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(ana, num, rtol=1e-5, atol=1e-7)
+
+
+def test_partial_gradient_over_all_keys_is_the_full_gradient():
+    r = _rng(81)
+    q, k, v, do = (r.standard_normal((2, 7, 4)) for _ in range(4))
+    o, lse = attn_fwd_ref(q, k, v, 0.5, True)
+    for a, b in zip(attn_bwd_partial_ref(q, k, v, o, do, lse, 0.5, True), attn_bwd_ref(q, k, v, do, 0.5, True)):
+        np.testing.assert_allclose(a, b, atol=1e-13)
+
+
+def test_partial_gradient_needs_the_full_row_statistics():
+    # with the chunk's own (O, LSE) instead of the full rows' the partial
+    # gradients do not add up: the sum over chunks is right only with the
+    # merged statistics
+    r = _rng(82)
+    q, k, v, do = (r.standard_normal((6, 3)) for _ in range(4))
+    o, lse = attn_fwd_ref(q, k, v, 0.7)
+    full = attn_bwd_ref(q, k, v, do, 0.7)
+    parts = [attn_bwd_partial_ref(q, k[c], v[c], o, do, lse, 0.7) for c in (slice(0, 2), slice(2, 6))]
+    np.testing.assert_allclose(parts[0][0] + parts[1][0], full[0], atol=1e-13)
+    np.testing.assert_allclose(np.concatenate([parts[0][1], parts[1][1]]), full[1], atol=1e-13)
+    np.testing.assert_allclose(np.concatenate([parts[0][2], parts[1][2]]), full[2], atol=1e-13)
+    o0, l0 = attn_fwd_ref(q, k[:2], v[:2], 0.7)
+    wrong = attn_bwd_partial_ref(q, k[:2], v[:2], o0, do, l0, 0.7)
+    assert np.abs(wrong[2] - parts[0][2]).max() > 1e-3
