@@ -20,3 +20,13 @@ from .attention import (  # noqa: F401
     ring_fwd_ref,
     ring_bwd_ref,
 )
+from .fp8 import (  # noqa: F401
+    E4M3_MAX,
+    e4m3_round_ref,
+    hadamard_ref,
+    rotate_ref,
+    quantize_rows_ref,
+    quantize_cols_ref,
+    fp8_inputs_ref,
+    fp8_attn_fwd_ref,
+)

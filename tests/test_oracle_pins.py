@@ -572,3 +572,134 @@ def test_partial_gradient_needs_the_full_row_statistics():
     o0, l0 = attn_fwd_ref(q, k[:2], v[:2], 0.7)
     wrong = attn_bwd_partial_ref(q, k[:2], v[:2], o0, do, l0, 0.7)
     assert np.abs(wrong[2] - parts[0][2]).max() > 1e-3
+
+
+# ---------------------------------------------------------------- FP8 forward
+
+from oracle import (E4M3_MAX, e4m3_round_ref, fp8_attn_fwd_ref, fp8_inputs_ref,  # noqa: E402
+                    hadamard_ref, quantize_cols_ref, quantize_rows_ref, rotate_ref)
+
+
+def _e4m3_table():
+    """Every non-negative finite e4m3 value with its code (exponent bias 7,
+    3 mantissa bits; exponent 0 = subnormal; code 0x7f is NaN)."""
+    out = []
+    for code in range(0x7f):
+        e, m = code >> 3, code & 7
+        val = m * 2.0 ** -9 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7)
+        out.append((val, code))
+    return out
+
+
+def test_e4m3_rounding_is_exhaustive_nearest_ties_to_even():
+    table = _e4m3_table()
+    vals = np.array([v for v, _ in table])
+    codes = np.array([c for _, c in table])
+    assert vals.max() == E4M3_MAX == 448.0
+    r = _rng(91)
+    x = np.concatenate([r.uniform(0, 448, 3000), np.exp2(r.uniform(-12, 8.8, 3000)),
+                        (vals[:-1] + vals[1:]) / 2,           # every midpoint: a tie
+                        vals])
+    x = x[x <= 448.0]
+    got = e4m3_round_ref(x)
+    for xi, gi in zip(x, got):
+        dist = np.abs(vals - xi)
+        best = np.flatnonzero(dist == dist.min())
+        if len(best) > 1:                                      # tie: even mantissa code
+            best = [b for b in best if codes[b] % 2 == 0]
+        assert gi == vals[best[0]], (xi, gi, vals[best[0]])
+    np.testing.assert_array_equal(e4m3_round_ref(-x), -got)
+
+
+def test_e4m3_rounding_matches_torch_float8_cast_and_saturates():
+    r = _rng(92)
+    x = np.concatenate([r.standard_normal(5000) * 50, r.standard_normal(5000) * 0.01]).astype(np.float32)
+    x = x[np.abs(x) <= 448]
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).double().numpy()
+    np.testing.assert_array_equal(e4m3_round_ref(x), want)
+    # beyond the largest finite value the oracle saturates (satfinite)
+    np.testing.assert_array_equal(e4m3_round_ref([464.0, 500.0, 1e6, -1e6]), [448.0, 448.0, 448.0, -448.0])
+
+
+def test_hadamard_is_sylvester_and_orthogonal():
+    import scipy.linalg
+    for d in (1, 2, 8, 64, 128):
+        h = hadamard_ref(d)
+        np.testing.assert_array_equal(h, scipy.linalg.hadamard(d))
+        np.testing.assert_array_equal(h @ h.T, d * np.eye(d))
+    with pytest.raises(ValueError):
+        hadamard_ref(96)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_fast_rotation_equals_the_matrix_product(d):
+    r = _rng(93 + d)
+    x = r.standard_normal((3, 50, d)).astype(np.float32)
+    s = r.choice([-1.0, 1.0], d)
+    y = rotate_ref(x, s)
+    assert y.dtype == np.float32
+    want = x.astype(np.float64) @ (np.diag(s) @ hadamard_ref(d)) / np.sqrt(d)
+    np.testing.assert_allclose(y, want, rtol=0, atol=2e-6 * np.abs(x).max() * np.sqrt(d))
+    # orthogonal: norms and inner products are kept
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-5)
+    k = r.standard_normal((3, 40, d)).astype(np.float32)
+    np.testing.assert_allclose(y @ np.swapaxes(rotate_ref(k, s), -1, -2), x @ np.swapaxes(k, -1, -2),
+                               atol=1e-3)
+
+
+def test_row_block_and_channel_quantisation():
+    r = _rng(94)
+    x = (r.standard_normal((2, 300, 16)) * np.array([1.0, 10.0])[:, None, None]).astype(np.float32)
+    x[1, 128:256] = 0.0                                        # an all-zero block
+    vals, sc = quantize_rows_ref(x)
+    assert sc.shape == (2, 3) and sc.dtype == np.float32
+    for h in range(2):
+        for b in range(3):
+            blk = x[h, 128 * b:128 * (b + 1)]
+            amax = np.float32(np.abs(blk).max())
+            if amax == 0:
+                assert sc[h, b] == 1.0 and not vals[h, 128 * b:128 * (b + 1)].any()
+                continue
+            assert sc[h, b] == amax / np.float32(448.0)
+            v = vals[h, 128 * b:128 * (b + 1)]
+            assert np.abs(v).max() == 448.0                    # the largest element maps to the top code
+            np.testing.assert_array_equal(v, e4m3_round_ref(blk / sc[h, b]))
+            # dequantised values within half an e4m3 step (2^-4 relative) or a subnormal step
+            err = np.abs(v * np.float64(sc[h, b]) - blk)
+            assert np.all(err <= np.maximum(np.abs(blk) * 2.0 ** -4, 2.0 ** -10 * float(sc[h, b])) * (1 + 1e-6))
+    cv, cs = quantize_cols_ref(x)
+    assert cs.shape == (2, 16)
+    np.testing.assert_array_equal(cs, np.where(np.abs(x).max(axis=1) > 0, np.abs(x).max(axis=1) / np.float32(448), 1))
+    assert np.all(np.abs(cv).max(axis=1)[np.abs(x).max(axis=1) > 0] == 448.0)
+
+
+def test_fp8_attention_of_exactly_representable_inputs_is_attention():
+    # entries in {0, +-1, +-2, +-4}, each block and channel holding a 4: every
+    # value is a code (112, 224 or 448) times the scale 4/448, so only the
+    # float32 rounding of the scale separates the result from exact attention
+    r = _rng(95)
+    q, k, v = (r.choice([0.0, 1.0, -1.0, 2.0, -2.0, 4.0, -4.0], (2, 256, 8)) for _ in range(3))
+    for x in (q, k, v):
+        x[:, ::128, :] = 4.0
+        x[:, :, 0] = np.where(np.arange(256) == 5, 4.0, x[:, :, 0])
+    o, lse = fp8_attn_fwd_ref(q, k, v, 0.3, True)
+    o2, lse2 = attn_fwd_ref(q, k, v, 0.3, True)
+    np.testing.assert_allclose(o, o2, atol=1e-5)
+    np.testing.assert_allclose(lse, lse2, atol=1e-5)
+
+
+def test_rotation_lowers_fp8_error_on_outlier_channels():
+    # the pages' claim (lower error than plain FP8 when a few channels carry
+    # outliers), on the oracle's own quantised attention
+    r = _rng(96)
+    d = 64
+    q, k, v = (r.standard_normal((1, 512, d)) for _ in range(3))
+    q[..., :2] *= 30.0
+    k[..., :2] *= 30.0
+    s = r.choice([-1.0, 1.0], d)
+    exact, _ = attn_fwd_ref(q, k, v, d ** -0.5)
+    plain, _ = fp8_attn_fwd_ref(q, k, v, d ** -0.5)
+    rot, _ = fp8_attn_fwd_ref(q, k, v, d ** -0.5, signs=s)
+    e_plain = np.sqrt(np.mean((plain - exact) ** 2))
+    e_rot = np.sqrt(np.mean((rot - exact) ** 2))
+    assert e_rot < e_plain / 1.5, (e_rot, e_plain)
