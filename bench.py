@@ -49,6 +49,10 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-target", action="store_true")
     ap.add_argument("--no-memory", action="store_true")
+    ap.add_argument("--variant", default="dense", choices=["dense", "gqa", "blocksparse", "fp8"],
+                    help="dense attention (default); grouped-query attention with H/4 key/value heads; "
+                         "block-sparse attention with a seeded random 128x128 tile mask keeping half the tiles; "
+                         "the FP8 forward with incoherent processing (d = 128, forward only)")
     return ap.parse_args()
 
 
@@ -248,17 +252,68 @@ def run_native(args):
         ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-
-    def step():
-        fa.fa_fwd(g["q"], g["k"], g["v"], o, lse, scale=w.scale, causal=w.causal, stream=stream)
-        ev_mid.record(stream)
-        if w.backward:
-            fa.fa_bwd(g["q"], g["k"], g["v"], o, g["do"], lse, dq, dk, dv, ws, scale=w.scale,
-                      causal=w.causal, stream=stream)
-
-    launches_per_step = 1 + (3 if w.backward else 0)
     f_fwd = attn_fwd_flops(B, H, N, d, w.causal)
-    f_bwd = attn_bwd_flops(B, H, N, d, w.causal) if w.backward else 0.0
+    variant = {"name": args.variant}
+
+    if args.variant == "dense":
+        def step():
+            fa.fa_fwd(g["q"], g["k"], g["v"], o, lse, scale=w.scale, causal=w.causal, stream=stream)
+            ev_mid.record(stream)
+            if w.backward:
+                fa.fa_bwd(g["q"], g["k"], g["v"], o, g["do"], lse, dq, dk, dv, ws, scale=w.scale,
+                          causal=w.causal, stream=stream)
+    elif args.variant == "gqa":
+        # H query heads over H/4 key/value heads (the first H/4 heads of the
+        # drawn K and V); the FLOPs are those of H query heads
+        hkv = max(1, H // 4)
+        kg, vg = (g[n][:, :hkv].contiguous() for n in ("k", "v"))
+        variant["Hkv"] = hkv
+        if w.backward:
+            dk, dv = torch.empty_like(kg), torch.empty_like(vg)
+
+        def step():
+            fa.fa_fwd_gqa(g["q"], kg, vg, o, lse, scale=w.scale, causal=w.causal, stream=stream)
+            ev_mid.record(stream)
+            if w.backward:
+                fa.fa_bwd_gqa(g["q"], kg, vg, o, g["do"], lse, dq, dk, dv, ws, scale=w.scale,
+                              causal=w.causal, stream=stream)
+    elif args.variant == "fp8":
+        # FP8 forward (rotation + block scales + e4m3 products), forward only;
+        # the step includes the quantisation of Q, K, V
+        if d != 128:
+            raise SystemExit("the fp8 variant needs a d = 128 workload")
+        g_signs = (torch.randint(0, 2, (128,), generator=torch.Generator().manual_seed(77)) * 2 - 1).float().to(dev)
+        ws8 = torch.empty(fa.fa_fwd_fp8_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+        variant.update(forward_only=True, operands="e4m3", rotation="random-sign Hadamard")
+
+        def step():
+            fa.fa_fwd_fp8(g["q"], g["k"], g["v"], g_signs, o, lse, ws8, scale=w.scale, causal=w.causal,
+                          stream=stream)
+            ev_mid.record(stream)
+    else:
+        # block-sparse: per head, each 128x128 tile kept with probability 1/2
+        # (seeded); FLOPs count only the (query, key) pairs actually attended
+        import numpy as np
+        nb = (N + 127) // 128
+        rng = np.random.default_rng(1234 + rank)
+        mask_np = (rng.random((B, H, nb, nb)) < 0.5).astype(np.uint8)
+        mask = torch.from_numpy(mask_np).to(dev)
+        kept = _attended_pairs(mask_np, N, w.causal)
+        dense_pairs = B * H * (N * N / 2.0 if w.causal else float(N * N))
+        f_fwd = f_fwd * kept / dense_pairs
+        variant.update(tile_density=float(mask_np.mean()), attended_fraction=kept / (B * H * float(N * N)))
+
+        def step():
+            fa.fa_fwd_blocksparse(g["q"], g["k"], g["v"], mask, o, lse, scale=w.scale, causal=w.causal,
+                                  stream=stream)
+            ev_mid.record(stream)
+            if w.backward:
+                fa.fa_bwd_blocksparse(g["q"], g["k"], g["v"], o, g["do"], lse, mask, dq, dk, dv, ws,
+                                      scale=w.scale, causal=w.causal, stream=stream)
+
+    with_bwd = w.backward and args.variant != "fp8"
+    launches_per_step = (4 if args.variant == "fp8" else 1) + (3 if with_bwd else 0)
+    f_bwd = 2.5 * f_fwd if with_bwd else 0.0
     flops = f_fwd + f_bwd
 
     ev_mid = torch.cuda.Event(enable_timing=True)
@@ -296,42 +351,49 @@ def run_native(args):
 
     # dominant kernel (the backward launch group when present, else the forward)
     peaks = _peaks()
-    if w.backward:
+    # FP8 products run at twice the 16-bit rate (the recipe's nominal 4.5 vs
+    # 2.25 PFLOP/s): their peak is the measured bf16 peak times 2
+    dt_ratio = 2.0 if args.variant == "fp8" else 1.0
+    if with_bwd:
         dom_ms, dom_flops, dom_name = statistics.mean(bwd_ms), f_bwd, "fa_bwd (prep + main + dQ convert launches)"
     else:
-        dom_ms, dom_flops, dom_name = statistics.mean(fwd_ms), f_fwd, "fa_fwd_kernel"
+        dom_ms, dom_flops, dom_name = statistics.mean(fwd_ms), f_fwd, \
+            "fa_fwd_fp8 (quantise + fa_fwd_kernel FP8)" if args.variant == "fp8" else "fa_fwd_kernel"
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": _ncu_traffic(w.name, dom_name),
-                "peak_source": f"{peaks['source']} bf16 burst", "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+    peak = peaks["bf16_tflops"] * dt_ratio
+    roofline = {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": _ncu_traffic(w.name, dom_name) if args.variant == "dense" else None,
+                "peak_source": f"{peaks['source']} bf16 burst" + (" x 2 (fp8 / bf16 nominal)" if dt_ratio != 1 else ""),
+                "frac_of_sustained": achieved / (peaks["bf16_tflops_sustained"] * dt_ratio),
                 "fwd_tflops": f_fwd / (statistics.mean(fwd_ms) * 1e-3) / 1e12,
-                "bwd_tflops": (f_bwd / (statistics.mean(bwd_ms) * 1e-3) / 1e12) if w.backward else None}
+                "bwd_tflops": (f_bwd / (statistics.mean(bwd_ms) * 1e-3) / 1e12) if with_bwd else None}
 
     # end to end through the public API: pinned host inputs -> device -> step -> host
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.variant == "dense":
         e2e = _e2e(fa, torch, w, x, dev, stream, flops, world, args)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
-        "config": _config(w, world), "roofline": roofline, "e2e": e2e,
+        "vs_baseline": None, "dtype": "e4m3 products, " + w.dtype + " in/out" if args.variant == "fp8" else w.dtype, "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
+        "config": dict(_config(w, world), variant=variant), "roofline": roofline, "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
-        "fwd_ms": statistics.mean(fwd_ms), "bwd_ms": statistics.mean(bwd_ms) if w.backward else None,
+        "fwd_ms": statistics.mean(fwd_ms), "bwd_ms": statistics.mean(bwd_ms) if with_bwd else None,
         "pct_of_peak": {"measured_burst": value / world / peaks["bf16_tflops"],
                         "measured_sustained": value / world / peaks["bf16_tflops_sustained"],
                         "datasheet_2250": value / world / 2250.0},
     }
-    if not args.no_memory and rank == 0:
+    if not args.no_memory and rank == 0 and args.variant == "dense":
         line["memory"] = _memory_vs_n(fa, torch, dev, stream)
     line["context"] = {
         "note": "the pages' own figures on other hardware; not targets",
         "fa2_a100_frac_of_peak": 0.70, "fa1_a100_frac_of_peak": 0.35,
         "source": "marketmaker.cc, FA2 section (A100 theoretical peak FLOPs)"}
-    if not args.no_target and w.name != TARGET_WORKLOAD:
-        line["north_star_target"] = _target_fwd(fa, torch, dev, stream, flush, peaks, args)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if not args.no_target and w.name != TARGET_WORKLOAD and args.variant == "dense":
+        line["target_fwd_d128_n8192_nc"] = _target_fwd(fa, torch, dev, stream, flush, peaks, args)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.variant == "dense":
         tf, heads, el = _oracle_sample(w, 12.0)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": _cpu_threads(), "kind": "oracle",
                                 "sample": f"{heads} whole (b,h) heads of {w.name}, fp64 forward"
@@ -342,6 +404,19 @@ def run_native(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def _attended_pairs(mask, N, causal):
+    """(query, key) pairs a block-sparse mask [B, H, nb, nb] leaves attended
+    (and, when causal, with key <= query), summed over heads."""
+    import numpy as np
+    nb = mask.shape[-1]
+    rows = np.minimum((np.arange(nb) + 1) * 128, N) - np.arange(nb) * 128      # queries per block
+    cnt = np.outer(rows, rows).astype(np.float64)                                # pairs per tile
+    if causal:
+        cnt = np.where(np.arange(nb)[None, :] < np.arange(nb)[:, None], cnt, 0.0)
+        cnt[np.arange(nb), np.arange(nb)] = rows * (rows + 1) / 2.0               # diagonal tiles
+    return float((mask.astype(np.float64) * cnt).sum())
 
 
 def _memory_vs_n(fa, torch, dev, stream):

@@ -27,6 +27,12 @@ __all__ = [
     "fa_bwd_gqa",
     "fa_fwd_blocksparse",
     "fa_bwd_blocksparse",
+    "fa_fwd_fp8_workspace_size",
+    "fa_fp8_quantize",
+    "fa_fwd_fp8",
+    "fa_merge",
+    "fa_grad_accumulate",
+    "fa_convert",
     "fa_status_string",
     "fa_last_device_status",
     "fa_debug_set_wait_limit_ms",
@@ -74,6 +80,13 @@ _SIGNATURES = {
                                     _c_int, _c_float, _c_int, _c_int, _vp]),
     "fa_bwd_blocksparse": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_longlong, _vp, _vp, _vp, _vp,
                                     _sz, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _vp]),
+    "fa_fwd_fp8_workspace_size": (_sz, [_c_int, _c_int, _c_int, _c_int]),
+    "fa_fp8_quantize": (_c_int, [_vp, _vp, _vp, _vp, _vp, _sz, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
+    "fa_fwd_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _c_int, _c_int, _c_int, _c_int, _c_float,
+                            _c_int, _c_int, _vp]),
+    "fa_merge": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, ctypes.c_longlong, _c_int, _vp]),
+    "fa_grad_accumulate": (_c_int, [_vp, _vp, ctypes.c_longlong, _c_int, _vp]),
+    "fa_convert": (_c_int, [_vp, _vp, ctypes.c_longlong, _c_int, _vp]),
     "fa_bwd_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _vp]),
     "fa_status_string": (ctypes.c_char_p, [_c_int]),
@@ -418,3 +431,133 @@ def fa_bwd_blocksparse(q, k, v, o, do, lse, block_mask, dq=None, dk=None, dv=Non
     if st != FA_OK:
         raise FAError(st, "fa_bwd_blocksparse")
     return dq, dk, dv
+
+
+def _dense_cuda(name, t, dtypes):
+    torch = _torch()
+    if not t.is_cuda or not t.is_contiguous() or t.dtype not in dtypes:
+        raise ValueError(f"{name} must be a contiguous CUDA tensor of type {dtypes}")
+
+
+def fa_merge(o, lse, o_part, lse_part, out=None, stream=None):
+    """In place: (o, lse) <- merge of two partial results over disjoint key
+    sets.  o, o_part fp32 [..., n, d]; lse, lse_part fp32 [..., n]; ``out``
+    (optional, bf16/fp16, shape of o) receives the merged O as well."""
+    torch = _torch()
+    for name, t in (("o", o), ("o_part", o_part)):
+        _dense_cuda(name, t, (torch.float32,))
+    for name, t in (("lse", lse), ("lse_part", lse_part)):
+        _dense_cuda(name, t, (torch.float32,))
+    if o_part.shape != o.shape or lse.shape != o.shape[:-1] or lse_part.shape != lse.shape:
+        raise ValueError("fa_merge: shapes of o, o_part, lse, lse_part disagree")
+    code = -1
+    if out is not None:
+        _dense_cuda("out", out, (torch.bfloat16, torch.float16))
+        if out.shape != o.shape:
+            raise ValueError("fa_merge: out must have the shape of o")
+        code = FA_BF16 if out.dtype == torch.bfloat16 else FA_FP16
+    d = o.shape[-1]
+    st = load_library().fa_merge(o.data_ptr(), lse.data_ptr(), o_part.data_ptr(), lse_part.data_ptr(),
+                                 out.data_ptr() if out is not None else None, code, lse.numel(), d,
+                                 _stream_handle(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_merge")
+    return o, lse
+
+
+def fa_grad_accumulate(acc, src, stream=None):
+    """In place: acc (fp32) += src (bf16/fp16), elementwise, same shape."""
+    torch = _torch()
+    _dense_cuda("acc", acc, (torch.float32,))
+    _dense_cuda("src", src, (torch.bfloat16, torch.float16))
+    if acc.shape != src.shape:
+        raise ValueError("fa_grad_accumulate: shapes differ")
+    st = load_library().fa_grad_accumulate(acc.data_ptr(), src.data_ptr(), acc.numel(),
+                                           FA_BF16 if src.dtype == torch.bfloat16 else FA_FP16,
+                                           _stream_handle(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_grad_accumulate")
+    return acc
+
+
+def fa_convert(src, dtype=None, out=None, stream=None):
+    """fp32 -> bf16/fp16 (round to nearest even) on the device."""
+    torch = _torch()
+    _dense_cuda("src", src, (torch.float32,))
+    if out is None:
+        out = torch.empty(src.shape, dtype=dtype or torch.bfloat16, device=src.device)
+    _dense_cuda("out", out, (torch.bfloat16, torch.float16))
+    if out.shape != src.shape:
+        raise ValueError("fa_convert: shapes differ")
+    st = load_library().fa_convert(out.data_ptr(), src.data_ptr(), src.numel(),
+                                   FA_BF16 if out.dtype == torch.bfloat16 else FA_FP16, _stream_handle(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_convert")
+    return out
+
+
+def fa_fwd_fp8_workspace_size(B: int, H: int, N: int, d: int = 128) -> int:
+    return int(load_library().fa_fwd_fp8_workspace_size(B, H, N, d))
+
+
+def _fp8_views(ws, B, H, N):
+    """Views of the FP8 workspace's parts (layout of fa_fwd_fp8_workspace_size)."""
+    torch = _torch()
+    bh, nb = B * H, (N + 127) // 128
+    n_pad = nb * 128
+    up = lambda x: (x + 255) // 256 * 256
+    off, out = 0, {}
+    for name, n, dt, shape in (("q8", bh * n_pad * 128, torch.uint8, (B, H, n_pad, 128)),
+                               ("k8", bh * n_pad * 128, torch.uint8, (B, H, n_pad, 128)),
+                               ("v8t", bh * n_pad * 128, torch.uint8, (B, H, 128, n_pad)),
+                               ("sq", bh * nb * 4, torch.float32, (B, H, nb)),
+                               ("sk", bh * nb * 4, torch.float32, (B, H, nb)),
+                               ("sv", bh * 128 * 4, torch.float32, (B, H, 128))):
+        out[name] = ws[off:off + n].view(dt).view(shape)
+        off += up(n)
+    return out
+
+
+def fa_fp8_quantize(q, k, v, signs=None, workspace=None, stream=None):
+    """Rotation (when ``signs`` is given), scales and e4m3 codes of the FP8
+    forward.  Returns a dict of views into the workspace: q8, k8 [B,H,n_pad,128]
+    and v8t [B,H,128,n_pad] (uint8 e4m3 bits), sq, sk [B,H,nb], sv [B,H,128]."""
+    torch = _torch()
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_bhnd(name, t, None if name == "q" else q)
+    B, H, N, d = q.shape
+    if workspace is None:
+        workspace = torch.empty(fa_fwd_fp8_workspace_size(B, H, N, d), dtype=torch.uint8, device=q.device)
+    st = load_library().fa_fp8_quantize(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                        signs.data_ptr() if signs is not None else None, workspace.data_ptr(),
+                                        workspace.numel(), B, H, N, d, _dtype_code(q, q), _stream_handle(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_fp8_quantize")
+    return _fp8_views(workspace, B, H, N)
+
+
+def fa_fwd_fp8(q, k, v, signs=None, o=None, lse=None, workspace=None, scale: Optional[float] = None,
+               causal: bool = False, stream=None, o_fp32: bool = False):
+    """FP8 forward (head dim 128) with incoherent processing when ``signs``
+    (CUDA float32 [128] of +-1) is given.  Returns (O, LSE)."""
+    torch = _torch()
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_bhnd(name, t, None if name == "q" else q)
+    B, H, N, d = q.shape
+    if signs is not None and (not signs.is_cuda or signs.dtype != torch.float32 or signs.numel() != d):
+        raise ValueError("signs must be a CUDA float32 tensor of d entries")
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    if o is None:
+        o = torch.empty(q.shape, dtype=torch.float32 if o_fp32 else q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(1, fa_fwd_fp8_workspace_size(B, H, N, d)), dtype=torch.uint8, device=q.device)
+    st = load_library().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                   signs.data_ptr() if signs is not None else None, workspace.data_ptr(),
+                                   workspace.numel(), B, H, N, d, float(scale), int(bool(causal)),
+                                   _dtype_code(q, o), _stream_handle(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd_fp8")
+    return o, lse

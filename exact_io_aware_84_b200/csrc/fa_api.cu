@@ -83,6 +83,55 @@ int device_info(DeviceInfo* out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// 8-bit [outer][rows][inner] tensor, box = 128 inner x 128 rows, 128-byte
+// swizzle (the FP8 operands: inner = 128 bytes of a row).
+int encode_u8_map(CUtensorMap* m, const void* ptr, int outer, int rows, int inner) {
+  auto fn = encode_fn();
+  if (!fn) return FA_ERR_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)outer};
+  cuuint64_t strides[2] = {(cuuint64_t)inner, (cuuint64_t)rows * inner};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// Layout of the FP8 forward's workspace (each part 256-byte aligned).
+struct Fp8Layout {
+  size_t q8, k8, v8t, sq, sk, sv, vamax, total;
+};
+Fp8Layout fp8_layout(int B, int H, int N) {
+  const size_t bh = (size_t)B * H;
+  const size_t nb = ((size_t)N + 127) / 128, n_pad = nb * 128;
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  Fp8Layout l;
+  l.q8 = 0;
+  l.k8 = l.q8 + up(bh * n_pad * 128);
+  l.v8t = l.k8 + up(bh * n_pad * 128);
+  l.sq = l.v8t + up(bh * n_pad * 128);
+  l.sk = l.sq + up(bh * nb * 4);
+  l.sv = l.sk + up(bh * nb * 4);
+  l.vamax = l.sv + up(bh * 128 * 4);
+  l.total = l.vamax + up(bh * 128 * 4);
+  return l;
+}
+
+Fp8Buffers fp8_buffers(void* ws, int B, int H, int N) {
+  const Fp8Layout l = fp8_layout(B, H, N);
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  Fp8Buffers f;
+  f.q8 = b + l.q8;
+  f.k8 = b + l.k8;
+  f.v8t = b + l.v8t;
+  f.sq = reinterpret_cast<float*>(b + l.sq);
+  f.sk = reinterpret_cast<float*>(b + l.sk);
+  f.sv = reinterpret_cast<float*>(b + l.sv);
+  f.vamax = reinterpret_cast<unsigned*>(b + l.vamax);
+  return f;
+}
+
 int check_common(int B, int H, int N, int d, float scale, int dtype) {
   if (B <= 0 || H <= 0 || N <= 0) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || scale > 3.0e38f) return FA_ERR_INVALID_ARG;
@@ -298,6 +347,119 @@ int fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* 
   if (!block_mask) return FA_ERR_INVALID_ARG;
   return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, H, N, d, scale, causal,
                   dtype, stream, block_mask, mask_head_stride);
+}
+
+size_t fa_fwd_fp8_workspace_size(int B, int H, int N, int d) {
+  if (check_common(B, H, N, d, 1.0f, FA_BF16) != FA_OK || d != 128) return 0;
+  return fp8_layout(B, H, N).total;
+}
+
+static int fp8_prep(const void* q, const void* k, const void* v, const float* signs, void* workspace,
+                    size_t workspace_bytes, int B, int H, int N, int d, int dtype, void* stream) {
+  if (!q || !k || !v) return FA_ERR_INVALID_ARG;
+  int st = check_common(B, H, N, d, 1.0f, dtype);
+  if (st != FA_OK) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(workspace)) return FA_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < fp8_layout(B, H, N).total) return FA_ERR_WORKSPACE;
+  DeviceInfo di;
+  if ((st = device_info(&di)) != FA_OK) return st;
+  const bool bf16 = dtype == FA_BF16 || dtype == FA_BF16_O_F32;
+  cudaError_t e = launch_fp8_prep(bf16, q, k, v, signs, fp8_buffers(workspace, B, H, N), B * H, N,
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* signs, void* workspace,
+                    size_t workspace_bytes, int B, int H, int N, int d, int dtype, void* stream) {
+  return fp8_prep(q, k, v, signs, workspace, workspace_bytes, B, H, N, d, dtype, stream);
+}
+
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, const float* signs,
+               void* workspace, size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+               int dtype, void* stream) {
+  if (!o || !lse) return FA_ERR_INVALID_ARG;
+  int st = check_common(B, H, N, d, scale, dtype);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+  if ((st = fp8_prep(q, k, v, signs, workspace, workspace_bytes, B, H, N, d, dtype, stream)) != FA_OK) return st;
+  DeviceInfo di;
+  if ((st = device_info(&di)) != FA_OK) return st;
+  const bool bf16 = dtype == FA_BF16 || dtype == FA_BF16_O_F32;
+  const bool o32 = dtype == FA_BF16_O_F32 || dtype == FA_FP16_O_F32;
+  const int bh = B * H;
+  const int n_pad = (N + 127) / 128 * 128;
+  const Fp8Buffers fb = fp8_buffers(workspace, B, H, N);
+  CUtensorMap tq, tk, tvt;
+  if (encode_u8_map(&tq, fb.q8, bh, n_pad, 128) != FA_OK || encode_u8_map(&tk, fb.k8, bh, n_pad, 128) != FA_OK ||
+      encode_u8_map(&tvt, fb.v8t, bh, 128, n_pad) != FA_OK)
+    return FA_ERR_CUDA;
+  FwdParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.N = N;
+  p.bh = bh;
+  p.H = H;
+  p.group = 1;
+  p.n_kv = (N + kBlockN - 1) / kBlockN;
+  p.n_pairs = (N + 2 * kBlockM - 1) / (2 * kBlockM);
+  p.n_units = bh * p.n_pairs;
+  p.scale_log2 = scale * kLog2e;
+  p.wait_limit_ns = wait_limit_ns();
+  p.debug_flags = g_debug_flags.load();
+  p.fp8_sq = fb.sq;
+  p.fp8_sk = fb.sk;
+  p.fp8_sv = fb.sv;
+  if (!(p.status = status_ptr())) return FA_ERR_CUDA;
+  const int grid = p.n_units < di.sms ? p.n_units : di.sms;
+  cudaError_t e = launch_fwd_fp8(bf16, o32, causal != 0, tq, tk, tvt, p, grid, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_merge(float* o, float* lse, const float* o_part, const float* lse_part, void* out, int out_dtype,
+             long long rows, int d, void* stream) {
+  if (rows < 0) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (out_dtype < -1 || out_dtype > FA_FP16) return FA_ERR_UNSUPPORTED;
+  if (rows == 0) return FA_OK;
+  if (!o || !lse || !o_part || !lse_part || (out_dtype >= 0 && !out)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(o) | reinterpret_cast<uintptr_t>(o_part)) % 16 != 0 ||
+      (out_dtype >= 0 && reinterpret_cast<uintptr_t>(out) % 8 != 0))
+    return FA_ERR_MISALIGNED;
+  DeviceInfo di;
+  int st;
+  if ((st = device_info(&di)) != FA_OK) return st;
+  const int kind = out_dtype < 0 ? 0 : (out_dtype == FA_BF16 ? 1 : 2);
+  cudaError_t e = launch_merge(d, kind, o, lse, o_part, lse_part, out_dtype < 0 ? nullptr : out, rows, di.sms,
+                               static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_grad_accumulate(float* acc, const void* src, long long n, int src_dtype, void* stream) {
+  if (n < 0) return FA_ERR_INVALID_ARG;
+  if (src_dtype != FA_BF16 && src_dtype != FA_FP16) return FA_ERR_UNSUPPORTED;
+  if (n == 0) return FA_OK;
+  if (!acc || !src) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(acc) | reinterpret_cast<uintptr_t>(src)) % 16 != 0) return FA_ERR_MISALIGNED;
+  DeviceInfo di;
+  int st;
+  if ((st = device_info(&di)) != FA_OK) return st;
+  cudaError_t e = launch_accumulate(src_dtype == FA_BF16, acc, src, n, di.sms, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_convert(void* dst, const float* src, long long n, int dst_dtype, void* stream) {
+  if (n < 0) return FA_ERR_INVALID_ARG;
+  if (dst_dtype != FA_BF16 && dst_dtype != FA_FP16) return FA_ERR_UNSUPPORTED;
+  if (n == 0) return FA_OK;
+  if (!dst || !src) return FA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(src) % 16 != 0 || reinterpret_cast<uintptr_t>(dst) % 8 != 0)
+    return FA_ERR_MISALIGNED;
+  DeviceInfo di;
+  int st;
+  if ((st = device_info(&di)) != FA_OK) return st;
+  cudaError_t e = launch_convert(dst_dtype == FA_BF16, dst, src, n, di.sms, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -127,13 +127,30 @@ __device__ __forceinline__ BUnit decode_bunit(int u, const BwdParams& p) {
 }
 
 // Whether iteration `it` of the unit is computed: its query block attends the
-// unit's key block (always when dense).
+// unit's key block (always when dense).  The mask bytes of 32 iterations are
+// fetched at once (independent loads) into a register window; a role that
+// walks its iterations forward loads each window once.
+struct IterWin {
+  int base = -32;
+  uint32_t bits = 0;
+};
 template <int D, bool SPARSE>
-__device__ __forceinline__ bool bactive(const BwdParams& p, const BUnit& bu, int it) {
+__device__ __forceinline__ bool bactive(IterWin& w, const BwdParams& p, const BUnit& bu, int it) {
   if constexpr (!SPARSE) return true;
   constexpr int BR = BwdLayout<D>::BR;
-  const int qblk = (bu.qtile(it) * BR) / kBlockN;
-  return p.bmask[(long long)bu.qbh(it) * p.bmask_stride + (long long)qblk * p.n_kv + bu.jk] != 0;
+  if (it < w.base || it >= w.base + 32) {
+    w.base = it & ~31;
+    w.bits = 0;
+#pragma unroll 8
+    for (int i = 0; i < 32; ++i) {
+      const int t = w.base + i;
+      if (t < bu.n_it) {
+        const int qblk = (bu.qtile(t) * BR) / kBlockN;
+        if (p.bmask[(long long)bu.qbh(t) * p.bmask_stride + (long long)qblk * p.n_kv + bu.jk] != 0) w.bits |= 1u << i;
+      }
+    }
+  }
+  return (w.bits >> (it - w.base)) & 1u;
 }
 
 // Tile of R rows x D columns stored as D/64 column blocks of R x 128 B (SW128).
@@ -236,8 +253,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tma_load_3d(base + L::kKOff + c * (kBlockN * 128), &tmK, BAR(L::kKVFull), c * 64, bu.jk * kBlockN, bu.kvbh, pol_kv);
           tma_load_3d(base + L::kVOff + c * (kBlockN * 128), &tmV, BAR(L::kKVFull), c * 64, bu.jk * kBlockN, bu.kvbh, pol_kv);
         }
+        IterWin iw;
         for (int it = 0; it < bu.n_it; ++it) {
-          if (!bactive<D, SPARSE>(p, bu, it)) continue;
+          if (!bactive<D, SPARSE>(iw, p, bu, it)) continue;
           const int i = bu.qtile(it), qbh = bu.qbh(it);
           const uint32_t st = q_iter % L::kStages, use = q_iter / L::kStages;
           if (use > 0 && !mbar_wait(BAR(L::kQEmpty + st), (use - 1) & 1, wc)) { ok = false; break; }
@@ -275,8 +293,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
         if (!mbar_wait(BAR(L::kKVFull), unit_iter & 1, wc)) { ok = false; break; }
         const uint32_t sK = base + L::kKOff, sV = base + L::kVOff;
+        IterWin iw;  // walks forward only: the scan for the next iteration leads
         int a0 = 0;  // first computed iteration (n_it when the key tile is attended by none)
-        while (a0 < bu.n_it && !bactive<D, SPARSE>(p, bu, a0)) ++a0;
+        while (a0 < bu.n_it && !bactive<D, SPARSE>(iw, p, bu, a0)) ++a0;
         // S^T for the first query tile
         if (a0 < bu.n_it) {
           const uint32_t st = q_iter % L::kStages;
@@ -288,14 +307,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mma_ss(tmem + L::kColS, kmaj<kBlockN>(sK, ks), kmaj<BR>(sQ, ks), idesc_s, ks > 0);
           tc_commit(BAR(L::kSFull));
         }
-        for (int it = a0; it < bu.n_it; ++it) {
-          if (!bactive<D, SPARSE>(p, bu, it)) continue;
+        for (int it = a0, nxt; it < bu.n_it; it = nxt) {  // active iterations only
           const uint32_t st = q_iter % L::kStages;
           const uint32_t sQ = base + L::kQOff + st * L::kQT;
           const uint32_t sDO = base + L::kDOOff + st * L::kQT;
           const uint32_t first = (it == a0);
-          int nxt = it + 1;
-          while (nxt < bu.n_it && !bactive<D, SPARSE>(p, bu, nxt)) ++nxt;
+          nxt = it + 1;
+          while (nxt < bu.n_it && !bactive<D, SPARSE>(iw, p, bu, nxt)) ++nxt;
           // dP^T = V_j dO_i^T   (the dP region's previous contents, dS^T of
           // tile i-1, were consumed by dK(i-1), issued earlier)
 #pragma unroll
@@ -321,13 +339,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               mma_ss(tmem + L::kColS, kmaj<kBlockN>(sK, ks), kmaj<BR>(sQ1, ks), idesc_s, ks > 0);
             tc_commit(BAR(L::kSFull));
           }
-          // dK += dS^T Q_i
           if (!mbar_wait(BAR(L::kDSFull), ds_cnt & 1, wc)) { ok = false; break; }
           ++ds_cnt;
           tc_fence_after();
+          // dK += dS^T Q_i
 #pragma unroll
           for (int ks = 0; ks < BR / 16; ++ks)
-            mma_ts(tmem + L::kColDK, tmem + L::kColDP + L::packed_col(ks), mnmaj<BR>(sQ, ks), idesc_acc, (!first || ks > 0) ? 1u : 0u);
+            mma_ts(tmem + L::kColDK, tmem + L::kColDP + L::packed_col(ks), mnmaj<BR>(sQ, ks), idesc_acc,
+                   (!first || ks > 0) ? 1u : 0u);
           // dQ_i (d=64) or dQ_i^T (d=128) from dS^T in shared memory
           if (dq_cnt > 0 && !mbar_wait(BAR(L::kDQEmpty), (dq_cnt - 1) & 1, wc)) { ok = false; break; }
           tc_fence_after();
@@ -341,8 +360,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           tc_commit(BAR(L::kDQFull));
           ++dq_cnt;
-          tc_commit(BAR(L::kQEmpty + st));   // Q_i, dO_i, LSE_i, D_i no longer read
           tc_commit(BAR(L::kDSEmpty));       // dS^T shared tile no longer read
+          tc_commit(BAR(L::kQEmpty + st));   // Q_i, dO_i, LSE_i, D_i no longer read
           ++q_iter;
         }
         if (!ok) break;
@@ -442,8 +461,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int key = bu.jk * kBlockN + key_in;
       const bool key_ok = key < p.N;
       int n_done = 0;  // iterations computed in this unit
+      IterWin iw;
       for (int it = 0; it < bu.n_it; ++it) {
-        if (!bactive<D, SPARSE>(p, bu, it)) continue;
+        if (!bactive<D, SPARSE>(iw, p, bu, it)) continue;
         const int i = bu.qtile(it);
         const uint32_t st = q_iter % L::kStages;
         ok = warp_all(mbar_wait(BAR(L::kQFull + st), (q_iter / L::kStages) & 1, wc));

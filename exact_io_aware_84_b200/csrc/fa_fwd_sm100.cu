@@ -60,10 +60,10 @@ static_assert(2 * kRegsSoftmax + kRegsOther <= 3 * kLaunchRegs, "register split 
 #define FA_FWD_SLOTS_D128 4
 #endif
 
-template <int D>
+template <int D, bool FP8 = false>
 struct FwdLayout {
-  static constexpr int kTile = kBlockM * D * 2;  // bytes of one 128 x D 16-bit tile
-  static constexpr int kSlots = (D == 128) ? FA_FWD_SLOTS_D128 : 8;  // K/V ring depth (tiles)
+  static constexpr int kTile = kBlockM * D * (FP8 ? 1 : 2);  // bytes of one 128 x D tile (16- or 8-bit)
+  static constexpr int kSlots = (D == 128 && !FP8) ? FA_FWD_SLOTS_D128 : 8;  // K/V ring depth (tiles)
   // Q buffers (each holds the unit's two query tiles).  A second buffer, to
   // prefetch the next unit's Q, measured no faster at d = 64 (the unit
   // boundary is dominated by the causal tile imbalance), so one is used.
@@ -106,19 +106,41 @@ struct UnitInfo {
   __device__ __forceinline__ int nbk(int t) const { return t ? nbk_1 : nbk_0; }
 };
 
-// Whether query block qblk of head bh attends key block kblk (dense: always).
-template <bool SPARSE>
-__device__ __forceinline__ bool tile_active(const FwdParams& p, int bh, int qblk, int kblk) {
-  if constexpr (!SPARSE) return true;
-  return p.bmask[(long long)bh * p.bmask_stride + (long long)qblk * p.n_kv + kblk] != 0;
+// Bits i < 32 of the result: whether row[j0 + i] (a mask byte) is non-zero,
+// for j0 + i < n.  The loads are independent, eight in flight at a time (the
+// producer and MMA warps run on 72 registers).
+__device__ __forceinline__ uint32_t mask_bits(const uint8_t* row, int j0, int n) {
+  uint32_t b = 0;
+#pragma unroll 8
+  for (int i = 0; i < 32; ++i)
+    if (j0 + i < n && row[j0 + i] != 0) b |= 1u << i;
+  return b;
 }
+
+// A 32-block window of a unit's block mask, kept in registers: bit i of w0 /
+// w1 says whether query tile 0 / 1 attends key block base + i (always 0 past
+// the tile's own nb).  Dense kernels never touch it.
+struct MaskWin {
+  int base = -32;
+  uint32_t w0 = 0, w1 = 0;
+  __device__ __forceinline__ void seek(const FwdParams& p, const UnitInfo& ui, int j) {
+    if (j >= base && j < base + 32) return;
+    base = j & ~31;
+    const uint8_t* m = p.bmask + (long long)ui.bh * p.bmask_stride;
+    w0 = mask_bits(m + (long long)(ui.r0_0 / kBlockM) * p.n_kv, base, ui.nb_0);
+    w1 = ui.nb_1 > 0 ? mask_bits(m + (long long)(ui.r0_1 / kBlockM) * p.n_kv, base, ui.nb_1) : 0u;
+  }
+  // query tile t attends key block j (j inside the window)
+  __device__ __forceinline__ bool tile(int t, int j) const { return ((t ? w1 : w0) >> (j - base)) & 1u; }
+};
+
 // Key block j is visited by the unit when either query tile attends it.
 template <bool SPARSE>
-__device__ __forceinline__ bool unit_block(const FwdParams& p, const UnitInfo& ui, int j) {
+__device__ __forceinline__ bool unit_block(const FwdParams& p, const UnitInfo& ui, MaskWin& w, int j) {
   if constexpr (!SPARSE) return j < ui.nmax;
-  const bool a0 = j < ui.nb_0 && tile_active<SPARSE>(p, ui.bh, ui.r0_0 / kBlockM, j);
-  const bool a1 = j < ui.nb_1 && tile_active<SPARSE>(p, ui.bh, ui.r0_1 / kBlockM, j);
-  return a0 || a1;
+  if (j >= ui.nmax) return false;
+  w.seek(p, ui, j);
+  return ((w.w0 | w.w1) >> (j - w.base)) & 1u;
 }
 
 template <bool CAUSAL, bool SPARSE>
@@ -143,11 +165,17 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams& p) {
   ui.nbk_1 = ui.nb_1;
   if constexpr (SPARSE) {
     ui.K = ui.nbk_0 = ui.nbk_1 = 0;
-    for (int j = 0; j < ui.nmax; ++j) {
-      if (!unit_block<SPARSE>(p, ui, j)) continue;
-      ++ui.K;
-      if (j < ui.nb_0) ++ui.nbk_0;
-      if (j < ui.nb_1) ++ui.nbk_1;
+    MaskWin w;
+    for (int j0 = 0; j0 < ui.nmax; j0 += 32) {
+      w.seek(p, ui, j0);
+      const uint32_t any = w.w0 | w.w1;
+      // visited blocks below each tile's own nb
+      const int n0 = ui.nb_0 - j0, n1 = ui.nb_1 - j0;
+      const uint32_t lo0 = n0 >= 32 ? 0xffffffffu : (n0 > 0 ? (1u << n0) - 1u : 0u);
+      const uint32_t lo1 = n1 >= 32 ? 0xffffffffu : (n1 > 0 ? (1u << n1) - 1u : 0u);
+      ui.K += __popc(any);
+      ui.nbk_0 += __popc(any & lo0);
+      ui.nbk_1 += __popc(any & lo1);
     }
   }
   return ui;
@@ -168,11 +196,22 @@ __device__ __forceinline__ uint64_t v_desc(uint32_t tile, int kstep) {
   return make_sdesc_sw128(tile + (uint32_t)kstep * 2048, kBlockN * 128, 1024);
 }
 
-template <int D, bool BF16, bool O32, bool CAUSAL, bool SPARSE>
+// FP8 variant (D = 128): Q, K and V^T arrive as float8 e4m3 codes; the two
+// products run as kind::f8f6f4 (K = 32 per instruction: the same 32-byte
+// steps through the 128-byte swizzled rows); S is dequantised with the
+// product of the Q-block and K-block scales folded into the exponent's
+// factor; P is rounded to e4m3 (four per tensor-memory column) for the P V
+// product, whose B operand is the transposed V tile (K-major: a row per head
+// dimension, 128 keys); the epilogue applies V's per-channel scales.  The
+// running sum l adds the unrounded P.  P stays within [0, 2^8] (the stale
+// max is at most 2^8 below the true one), inside e4m3's range of 448.
+template <int D, bool BF16, bool O32, bool CAUSAL, bool SPARSE, bool FP8 = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using L = FwdLayout<D>;
+  static_assert(!FP8 || (D == 128 && !SPARSE), "the FP8 variant is dense, head dim 128");
+  using L = FwdLayout<D, FP8>;
+  constexpr int kQKBoxes = FP8 ? 1 : D / 64;   // 128-byte column blocks per Q / K tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -234,20 +273,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int t = 0; t < 2; ++t) {
           if (ui.nb(t) == 0) continue;
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c)
+          for (int c = 0; c < kQKBoxes; ++c)
             tma_load_3d(base + L::kQOff + (qb * 2 + t) * L::kTile + c * (kBlockM * 128), &tmQ, BAR(L::kQFull + qb), c * 64,
                         ui.r0(t), ui.bh, pol_q);
         }
+        MaskWin mw;
         for (int j = 0; j < ui.nmax && ok; ++j) {
-          if (!unit_block<SPARSE>(p, ui, j)) continue;
+          if (!unit_block<SPARSE>(p, ui, mw, j)) continue;
           for (int kv = 0; kv < 2; ++kv, ++kv_iter) {
             const uint32_t slot = kv_iter % L::kSlots;
             const uint32_t use = kv_iter / L::kSlots;
             if (use > 0 && !mbar_wait(BAR(L::kKVEmpty + slot), (use - 1) & 1, wc)) { ok = false; break; }
             mbar_arrive_expect_tx(BAR(L::kKVFull + slot), L::kTile);
-            for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(base + L::kKVOff + slot * L::kTile + c * (kBlockN * 128), kv ? &tmV : &tmK,
-                          BAR(L::kKVFull + slot), c * 64, j * kBlockN, ui.kvbh, pol_kv);
+            if (FP8 && kv) {
+              // V^T tile: 128 head dims x 128 keys (x = key, y = dim)
+              tma_load_3d(base + L::kKVOff + slot * L::kTile, &tmV, BAR(L::kKVFull + slot), j * kBlockN, 0, ui.kvbh,
+                          pol_kv);
+            } else {
+              for (int c = 0; c < kQKBoxes; ++c)
+                tma_load_3d(base + L::kKVOff + slot * L::kTile + c * (kBlockN * 128), kv ? &tmV : &tmK,
+                            BAR(L::kKVFull + slot), c * 64, j * kBlockN, ui.kvbh, pol_kv);
+            }
           }
         }
       }
@@ -268,8 +314,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = make_idesc_f16(BF16, kBlockM, kBlockN, false, false);
-      constexpr uint32_t idesc_pv = make_idesc_f16(BF16, kBlockM, D, false, true);
+      // kind::f8f6f4 with e4m3 operands uses the same fields (format code 0)
+      constexpr uint32_t idesc_s = make_idesc_f16(FP8 ? false : BF16, kBlockM, kBlockN, false, false);
+      constexpr uint32_t idesc_pv = make_idesc_f16(FP8 ? false : BF16, kBlockM, D, false, !FP8);
       uint32_t kv_iter = 0, unit_iter = 0;
       uint32_t p_cnt0 = 0, p_cnt1 = 0, o_uses0 = 0, o_uses1 = 0;
       bool ok = true;
@@ -303,9 +350,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               if (!ok) continue;
               tc_fence_after();
               const uint32_t vt = base + L::kKVOff + (v_idx % L::kSlots) * L::kTile;
+              if constexpr (FP8) {
 #pragma unroll
-              for (int ks = 0; ks < kBlockN / 16; ++ks)
-                mma_ts(tmem + colO, tmem + colS + 8u * ks, v_desc(vt, ks), idesc_pv, (j > 1 || ks > 0) ? 1u : 0u);
+                for (int ks = 0; ks < kBlockN / 32; ++ks)
+                  mma_ts_f8(tmem + colO, tmem + colS + 8u * ks, kmajor_desc<128>(vt, ks), idesc_pv,
+                            (j > 1 || ks > 0) ? 1u : 0u);
+              } else {
+#pragma unroll
+                for (int ks = 0; ks < kBlockN / 16; ++ks)
+                  mma_ts(tmem + colO, tmem + colS + 8u * ks, v_desc(vt, ks), idesc_pv, (j > 1 || ks > 0) ? 1u : 0u);
+              }
               if (j == nbt) tc_commit(BAR(L::kOFull + t));
             }
             if (j < nbt) {
@@ -320,9 +374,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               // S_t = Q_t K_j^T
               const uint32_t qt = base + L::kQOff + (qb * 2 + t) * L::kTile;
               const uint32_t kt = base + L::kKVOff + (k_idx % L::kSlots) * L::kTile;
+              if constexpr (FP8) {
 #pragma unroll
-              for (int ks = 0; ks < D / 16; ++ks)
-                mma_ss(tmem + colS, kmajor_desc<D>(qt, ks), kmajor_desc<D>(kt, ks), idesc_s, ks > 0 ? 1u : 0u);
+                for (int ks = 0; ks < D / 32; ++ks)
+                  mma_ss_f8(tmem + colS, kmajor_desc<D>(qt, ks), kmajor_desc<D>(kt, ks), idesc_s, ks > 0 ? 1u : 0u);
+              } else {
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks)
+                  mma_ss(tmem + colS, kmajor_desc<D>(qt, ks), kmajor_desc<D>(kt, ks), idesc_s, ks > 0 ? 1u : 0u);
+              }
               tc_commit(BAR(L::kSFull + t));
             }
           }
@@ -361,10 +421,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const int nb = ui.nbk(t);                    // key blocks this tile visits
       const int row = ui.r0(t) + r_in;
       const int qblk = ui.r0(t) / kBlockM;
+      // FP8: the query block's dequantisation scale, folded into the factor
+      float sq_l2 = sl2;
+      if constexpr (FP8) sq_l2 = sl2 * p.fp8_sq[(size_t)ui.bh * p.n_kv + qblk];
       float m_run = -INFINITY, l_run = 0.f;        // m_run stays -inf until a key is seen
       int jb = -1;                                 // index of the current key block
+      MaskWin mw;
       for (int j = 0; j < nb; ++j) {
-        do { ++jb; } while (!unit_block<SPARSE>(p, ui, jb));
+        do { ++jb; } while (!unit_block<SPARSE>(p, ui, mw, jb));
         ok = warp_all(mbar_wait(BAR(L::kSFull + t), s_cnt & 1, wc));
         if (!ok) break;
         ++s_cnt;
@@ -377,10 +441,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(sr[c]);
         const int kbase = jb * kBlockN;
-        if (SPARSE && !tile_active<SPARSE>(p, ui.bh, qblk, jb)) {
-          // visited for the other query tile only: nothing of it is kept here
-#pragma unroll
-          for (int c = 0; c < kBlockN; ++c) s[c] = -INFINITY;
+        // Block-sparse: a block visited for the other query tile only keeps
+        // nothing here.  Its scores are left as they are (finite: no causal or
+        // ragged mask is applied to it) and dropped below through the row
+        // max and the exponent, which is cheaper in registers than masking.
+        const bool dead = SPARSE && !mw.tile(t, jb);
+        // factor from raw scores to log2 units (FP8: times both block scales)
+        float c_l2 = sl2;
+        if constexpr (FP8) c_l2 = sq_l2 * p.fp8_sk[(size_t)ui.kvbh * p.n_kv + jb];
+        if (dead) {
         } else if (CAUSAL && jb == qblk) {
 #pragma unroll
           for (int c = 0; c < kBlockN; ++c)
@@ -399,7 +468,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int a = 0; a < 8; ++a) pm[a] = fmax3(pm[a], s[c + a], s[c + a + 8]);
         const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
-        const float m_new = fmaxf(m_run, mx * sl2);
+        const float m_new = fmaxf(m_run, dead ? -INFINITY : mx * c_l2);
         // Until a row has seen a key, its O and l are zero: the first finite
         // max is taken as is, without a rescale.
         const bool fresh = m_run == -INFINITY;
@@ -428,22 +497,33 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
           }
         }
-        const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;  // -inf row: every P is 0
+        // -inf row: every P is 0.  Dead block: x = s * 0 - inf = -inf, P = 0.
+        const float neg_m = dead ? -INFINITY : (m_run == -INFINITY) ? 0.f : -m_run;
+        const float sl2x = dead ? 0.f : c_l2;
         float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int q = 0; q < kBlockN / 32; ++q) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float x0 = fmaf(s[32 * q + 2 * e], sl2, neg_m);
-            const float x1 = fmaf(s[32 * q + 2 * e + 1], sl2, neg_m);
+            const float x0 = fmaf(s[32 * q + 2 * e], sl2x, neg_m);
+            const float x1 = fmaf(s[32 * q + 2 * e + 1], sl2x, neg_m);
             const bool poly = (poly_pair_mask<D>() >> (e & 7)) & 1u;
             const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
             const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
             ps[e & 3] += p0 + p1;
-            pk[e] = pack2<BF16>(p0, p1);
+            if constexpr (FP8) {
+              // two e4m3 per 16 bits; element pairs (2e, 2e + 1) of 32 keys
+              const uint32_t h = pack_e4m3x2(p0, p1);
+              if (e & 1) pk[e >> 1] |= h << 16; else pk[e >> 1] = h;
+            } else {
+              pk[e] = pack2<BF16>(p0, p1);
+            }
           }
-          tmem_st16(tS + 16u * q, pk);
+          if constexpr (FP8)
+            tmem_st8(tS + 8u * q, pk);   // 32 keys = 8 columns of four e4m3
+          else
+            tmem_st16(tS + 16u * q, pk);
         }
         l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         tmem_wait_st();
@@ -474,6 +554,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+        if constexpr (FP8) {  // V's per-channel dequantisation scales
+          const float* svp = p.fp8_sv + (size_t)ui.kvbh * D + 32 * c;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * svp[e]);
         }
         if constexpr (O32) {
           if (in_range) {
@@ -547,7 +632,33 @@ cudaError_t launch_fwd_d(bool bf16, bool o32, bool causal, const CUtensorMap& tq
 
 }  // namespace
 
+template <bool BF16, bool O32, bool CAUSAL>
+cudaError_t launch_fwd_fp8_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tvt,
+                             const FwdParams& p, int grid, cudaStream_t st) {
+  auto kern = fa_fwd_kernel<128, BF16, O32, CAUSAL, false, true>;
+  constexpr int smem = FwdLayout<128, true>::kAlloc;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kFwdThreads, smem, st>>>(tq, tk, tvt, p);
+  return cudaGetLastError();
+}
+
 int fwd_threads() { return kFwdThreads; }
+int fwd_fp8_smem() { return FwdLayout<128, true>::kAlloc; }
+
+cudaError_t launch_fwd_fp8(bool bf16, bool o32, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
+                           const CUtensorMap& tvt, const FwdParams& p, int grid, cudaStream_t st) {
+  if (bf16) {
+    if (o32) return causal ? launch_fwd_fp8_t<true, true, true>(tq, tk, tvt, p, grid, st)
+                           : launch_fwd_fp8_t<true, true, false>(tq, tk, tvt, p, grid, st);
+    return causal ? launch_fwd_fp8_t<true, false, true>(tq, tk, tvt, p, grid, st)
+                  : launch_fwd_fp8_t<true, false, false>(tq, tk, tvt, p, grid, st);
+  }
+  if (o32) return causal ? launch_fwd_fp8_t<false, true, true>(tq, tk, tvt, p, grid, st)
+                         : launch_fwd_fp8_t<false, true, false>(tq, tk, tvt, p, grid, st);
+  return causal ? launch_fwd_fp8_t<false, false, true>(tq, tk, tvt, p, grid, st)
+                : launch_fwd_fp8_t<false, false, false>(tq, tk, tvt, p, grid, st);
+}
 
 cudaError_t launch_fwd(int d, bool bf16, bool o32, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const FwdParams& p, int grid, cudaStream_t st) {

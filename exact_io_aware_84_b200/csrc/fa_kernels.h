@@ -29,6 +29,23 @@ struct FwdParams {
   // head, head h at bmask + h * bmask_stride (stride 0 = one mask for all).
   const uint8_t* bmask;
   long long bmask_stride;
+  // FP8 variant only (d = 128): dequantisation scales, e4m3 codes in the
+  // tensor maps.  Q: [B*H][n_kv] per 128-row block; K: [B*Hkv][n_kv];
+  // V: [B*Hkv][128] per channel.
+  const float* fp8_sq;
+  const float* fp8_sk;
+  const float* fp8_sv;
+};
+
+// Device buffers of the FP8 forward's quantised operands (see fa_fp8.cu).
+struct Fp8Buffers {
+  uint8_t* q8;     // [B*H][n_pad][128] e4m3
+  uint8_t* k8;     // [B*H][n_pad][128] e4m3
+  uint8_t* v8t;    // [B*H][128][n_pad] e4m3 (transposed)
+  float* sq;       // [B*H][n_kv]
+  float* sk;       // [B*H][n_kv]
+  float* sv;       // [B*H][128]
+  unsigned* vamax; // [B*H][128] scratch: channel maxima (float bits)
 };
 
 struct BwdParams {
@@ -59,10 +76,23 @@ struct BwdParams {
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_fwd(int d, bool bf16, bool o32, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const FwdParams& p, int grid, cudaStream_t st);
+// FP8 forward (d = 128): e4m3 Q, K (K-major) and V^T tensor maps; `bf16`
+// selects the output type.
+cudaError_t launch_fwd_fp8(bool bf16, bool o32, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
+                           const CUtensorMap& tvt, const FwdParams& p, int grid, cudaStream_t st);
+cudaError_t launch_fp8_prep(bool bf16, const void* q, const void* k, const void* v, const float* signs,
+                            const Fp8Buffers& b, int bh, int N, cudaStream_t st);
+int fwd_fp8_smem();
 
 cudaError_t launch_bwd(int d, bool bf16, bool o32, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p, int grid,
                        cudaStream_t st);
+
+// Ring-attention helpers (fa_ring.cu).  out_kind: 0 none, 1 bf16, 2 fp16.
+cudaError_t launch_merge(int d, int out_kind, float* o, float* lse, const float* o_part, const float* lse_part,
+                         void* out, long long rows, int sms, cudaStream_t st);
+cudaError_t launch_accumulate(bool bf16, float* acc, const void* src, long long n, int sms, cudaStream_t st);
+cudaError_t launch_convert(bool bf16, void* dst, const float* src, long long n, int sms, cudaStream_t st);
 
 int fwd_threads();
 int bwd_threads();

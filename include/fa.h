@@ -186,6 +186,85 @@ int fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* 
                        void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
                        float scale, int causal, int dtype, void* stream);
 
+/*
+ * Ring attention (context parallelism) splits the sequence into one chunk per
+ * device; each device keeps its query chunk and computes attention block by
+ * block against the key/value chunks as they pass around a ring (ultralytics
+ * glossary "Flash Attention", "Flash Attention and related terms", ring
+ * attention).  The per-chunk attention is fa_fwd / fa_bwd on the chunk pair
+ * (fp32-O dtype codes for the partial forward; the merged O and LSE for the
+ * backward); the two calls below are the steps between chunks.  The ring
+ * schedule and the exchange live in the Python package (exact_io_aware_84_b200.ring).
+ *
+ * fa_merge: (o, lse) <- the combination of two partial results of the same
+ * rows over disjoint key sets:
+ *   LSE = ln(e^{LSE_a} + e^{LSE_b}),  O = e^{LSE_a - LSE} O_a + e^{LSE_b - LSE} O_b
+ * (the online-softmax recurrence of marketmaker.cc "Online softmax
+ * recurrence", one whole chunk at a time).  Rows where both LSEs are -inf
+ * give O = 0, LSE = -inf.
+ *   o, o_part     : device fp32 [rows][d], 16-byte aligned; o updated in place
+ *   lse, lse_part : device fp32 [rows]; lse updated in place
+ *   out           : optional device [rows][d] 16-bit copy of the merged O
+ *                   (8-byte aligned), written when out_dtype is FA_BF16 or
+ *                   FA_FP16; out_dtype = -1 writes none (out may be NULL)
+ *   rows          : number of rows (B*H*n for a [B,H,n,d] chunk); 0 is a no-op
+ *   d             : 64 or 128
+ * Errors: FA_ERR_INVALID_ARG (NULL pointer, rows < 0), FA_ERR_UNSUPPORTED (d,
+ * out_dtype), FA_ERR_MISALIGNED, FA_ERR_CUDA (launch).
+ *
+ * fa_grad_accumulate: acc[i] += src[i] for i < n, src 16-bit (FA_BF16 or
+ * FA_FP16), acc fp32; both device pointers 16-byte aligned.  Used to sum the
+ * per-chunk gradients of the ring backward in fp32.  Errors as fa_merge.
+ *
+ * fa_convert: dst[i] = src[i] rounded to nearest even in the 16-bit type
+ * dst_dtype (FA_BF16 or FA_FP16), i < n; src fp32 16-byte aligned, dst 8-byte
+ * aligned.  Writes the ring's fp32 results (O, dQ, dK, dV) out in the input
+ * type.  Errors as fa_merge.
+ */
+int fa_merge(float* o, float* lse, const float* o_part, const float* lse_part, void* out, int out_dtype,
+             long long rows, int d, void* stream);
+int fa_grad_accumulate(float* acc, const void* src, long long n, int src_dtype, void* stream);
+int fa_convert(void* dst, const float* src, long long n, int dst_dtype, void* stream);
+
+/*
+ * FP8 forward with incoherent processing (head dim 128).  FP8 attention is
+ * hurt by outliers; multiplying the vectors by a random orthogonal matrix
+ * before the block-wise quantisation spreads an outlier over all coordinates
+ * (marketmaker.cc "Flash Attention and the sequence-length problem", section
+ * "FA3: Hopper mechanics", item 3).  Here:
+ *   rotation  R = diag(signs) H / sqrt(128), H the Sylvester Hadamard matrix,
+ *             applied to Q and K only ((Q R)(K R)^T = Q K^T); signs = NULL
+ *             skips it (plain FP8);
+ *   format    float8 e4m3, round to nearest even, saturating at +-448;
+ *   scales    Q and K one per (head, 128-row block), V one per (head,
+ *             channel): scale = amax / 448 (1 if amax = 0), code = e4m3(x / scale);
+ *   products  S = Q8 K8^T and O = P8 V8 on the tensor cores in FP8 with fp32
+ *             accumulation; S is dequantised through the exponent's factor,
+ *             P rounded to e4m3 (l sums the unrounded P), O times V's channel
+ *             scales in the epilogue.
+ * This approximates attention; the error is that of the e4m3 rounding of Q,
+ * K, V (after the rotation) and of P.
+ *
+ * fa_fwd_fp8_workspace_size(B, H, N, 128): bytes of the caller-owned scratch
+ *   (0 for an unsupported d): Q8, K8 [B*H][n_pad][128] and V8^T
+ *   [B*H][128][n_pad] e4m3 (n_pad = ceil(N/128)*128), then the fp32 scales
+ *   sq, sk [B*H][ceil(N/128)] and sv [B*H][128], then [B*H][128] words of
+ *   scratch; each part starts on a 256-byte boundary, in that order.
+ * fa_fp8_quantize: only the preparation (rotation, scales, codes) into the
+ *   workspace; exposed so that the codes can be checked.
+ * fa_fwd_fp8: preparation + attention.  q, k, v: [B,H,N,128] 16-bit (dtype
+ *   FA_BF16 / FA_FP16, or the _O_F32 codes for a float32 O); o, lse as in
+ *   fa_fwd; signs: device float[128] of +-1 or NULL.  Errors: as fa_fwd, plus
+ *   FA_ERR_UNSUPPORTED for d != 128 and FA_ERR_WORKSPACE for a missing or
+ *   short workspace.
+ */
+size_t fa_fwd_fp8_workspace_size(int B, int H, int N, int d);
+int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* signs, void* workspace,
+                    size_t workspace_bytes, int B, int H, int N, int d, int dtype, void* stream);
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, const float* signs,
+               void* workspace, size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+               int dtype, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fa_status_string(int status);
 

@@ -136,3 +136,37 @@ def test_blocksparse_rejects_null_mask_and_negative_stride():
     assert lib.fa_fwd_blocksparse(p, p, p, p, p, p, -1, 1, 1, 128, 64, 0.125, 0, 0, None) == fa.FA_ERR_INVALID_ARG
     assert lib.fa_bwd_blocksparse(p, p, p, p, p, p, None, 0, p, p, p, p, 1 << 20, 1, 1, 128, 64, 0.125, 0, 0,
                                   None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_ring_helpers_argument_errors():
+    lib = fa.load_library()
+    p = 0x1000
+    # d, out type, sizes, pointers and alignment are checked before any launch
+    assert lib.fa_merge(p, p, p, p, None, -1, 10, 96, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_merge(p, p, p, p, None, 2, 10, 64, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_merge(p, p, p, p, None, -1, -1, 64, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_merge(p, p, p, p, None, -1, 0, 64, None) == fa.FA_OK
+    assert lib.fa_merge(p, p, None, p, None, -1, 4, 64, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_merge(p, p, p, p, None, 0, 4, 64, None) == fa.FA_ERR_INVALID_ARG      # out missing
+    assert lib.fa_merge(p + 4, p, p, p, None, -1, 4, 64, None) == fa.FA_ERR_MISALIGNED
+    assert lib.fa_merge(p, p, p, p, p + 2, 0, 4, 64, None) == fa.FA_ERR_MISALIGNED
+    assert lib.fa_grad_accumulate(p, p, 0, 0, None) == fa.FA_OK
+    assert lib.fa_grad_accumulate(p, p, 8, 2, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_grad_accumulate(p, p, -1, 0, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_grad_accumulate(p, p + 8, 8, 0, None) == fa.FA_ERR_MISALIGNED
+    assert lib.fa_convert(p, p, 0, 1, None) == fa.FA_OK
+    assert lib.fa_convert(p, p, 8, 3, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_convert(p + 4, p, 8, 0, None) == fa.FA_ERR_MISALIGNED
+    assert lib.fa_convert(None, p, 8, 0, None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_fp8_argument_errors():
+    lib = fa.load_library()
+    p = 0x1000
+    assert lib.fa_fwd_fp8_workspace_size(1, 1, 128, 64) == 0
+    assert lib.fa_fwd_fp8_workspace_size(1, 1, 128, 128) > 3 * 128 * 128
+    assert lib.fa_fwd_fp8(p, p, p, p, p, None, p, 1 << 30, 1, 1, 128, 64, 0.1, 0, 0, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_fwd_fp8(p, p, p, p, p, None, None, 0, 1, 1, 128, 128, 0.1, 0, 0, None) == fa.FA_ERR_WORKSPACE
+    assert lib.fa_fwd_fp8(p, p, p, p, p, None, p, 16, 1, 1, 128, 128, 0.1, 0, 0, None) == fa.FA_ERR_WORKSPACE
+    assert lib.fa_fwd_fp8(p, p, p, None, p, None, p, 1 << 30, 1, 1, 128, 128, 0.1, 0, 0, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_fp8_quantize(None, p, p, None, p, 1 << 30, 1, 1, 128, 128, 0, None) == fa.FA_ERR_INVALID_ARG
