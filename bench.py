@@ -49,10 +49,13 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-target", action="store_true")
     ap.add_argument("--no-memory", action="store_true")
-    ap.add_argument("--variant", default="dense", choices=["dense", "gqa", "blocksparse", "fp8"],
+    ap.add_argument("--variant", default="dense", choices=["dense", "gqa", "blocksparse", "fp8", "ring"],
                     help="dense attention (default); grouped-query attention with H/4 key/value heads; "
                          "block-sparse attention with a seeded random 128x128 tile mask keeping half the tiles; "
-                         "the FP8 forward with incoherent processing (d = 128, forward only)")
+                         "the FP8 forward with incoherent processing (d = 128, forward only); ring attention "
+                         "over --ring-size ranks emulated by host threads on this GPU (the ring's device work "
+                         "without the transfers)")
+    ap.add_argument("--ring-size", type=int, default=4)
     return ap.parse_args()
 
 
@@ -290,6 +293,38 @@ def run_native(args):
             fa.fa_fwd_fp8(g["q"], g["k"], g["v"], g_signs, o, lse, ws8, scale=w.scale, causal=w.causal,
                           stream=stream)
             ev_mid.record(stream)
+    elif args.variant == "ring":
+        # the sequence split into R chunks, one per emulated rank; every rank
+        # runs the ring forward, then the ring backward (merges, fp32
+        # accumulation and conversions included); same FLOPs as full attention
+        from exact_io_aware_84_b200.ring import ThreadRing, ring_attention_bwd, ring_attention_fwd
+        R = args.ring_size
+        if N % R:
+            raise SystemExit(f"N = {N} is not a multiple of the ring size {R}")
+        n = N // R
+        chunks = [{k: t[:, :, r * n:(r + 1) * n].contiguous() for k, t in g.items()} for r in range(R)]
+        ring = ThreadRing(R)
+        state = [None] * R
+        variant.update(ring_size=R, chunk=n, transfers="device copies on one GPU (no NVLink)")
+
+        def fwd_rank(r):
+            torch.cuda.set_device(dev)
+            c = chunks[r]
+            state[r] = ring_attention_fwd(c["q"], c["k"], c["v"], scale=w.scale, causal=w.causal,
+                                          comm=ring.comm(r))
+
+        def bwd_rank(r):
+            torch.cuda.set_device(dev)
+            c = chunks[r]
+            _, l_r, o32_r = state[r]
+            ring_attention_bwd(c["q"], c["k"], c["v"], o32_r, c["do"], l_r, scale=w.scale, causal=w.causal,
+                               comm=ring.comm(r))
+
+        def step():
+            ring.run(fwd_rank)
+            ev_mid.record(stream)
+            if w.backward:
+                ring.run(bwd_rank)
     else:
         # block-sparse: per head, each 128x128 tile kept with probability 1/2
         # (seeded); FLOPs count only the (query, key) pairs actually attended
@@ -313,6 +348,12 @@ def run_native(args):
 
     with_bwd = w.backward and args.variant != "fp8"
     launches_per_step = (4 if args.variant == "fp8" else 1) + (3 if with_bwd else 0)
+    if args.variant == "ring":
+        # per rank and step: forward 1 (+1 merge), backward 3 + 3 accumulates;
+        # per rank: 1 + 3 conversions (skipped chunk pairs launch nothing)
+        R = args.ring_size
+        pairs = R * (R + 1) // 2 if w.causal else R * R
+        launches_per_step = (pairs + (pairs - R) + R) + ((6 * pairs + 3 * R) if with_bwd else 0)
     f_bwd = 2.5 * f_fwd if with_bwd else 0.0
     flops = f_fwd + f_bwd
 

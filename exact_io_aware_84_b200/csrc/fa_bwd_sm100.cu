@@ -165,6 +165,13 @@ template <int R>
 __device__ __forceinline__ uint64_t mnmaj(uint32_t tile, int kstep) {
   return make_sdesc_sw128(tile + (uint32_t)kstep * 2048, R * 128, 1024);
 }
+// Byte offsets of K step `kstep` in the two views (for sdesc_advance: the MMA
+// issuer builds each descriptor once and steps it by these constants).
+template <int R>
+__host__ __device__ constexpr uint32_t kmaj_off(int kstep) {
+  return (uint32_t)(kstep >> 2) * (R * 128) + (uint32_t)(kstep & 3) * 32;
+}
+__host__ __device__ constexpr uint32_t mnmaj_off(int kstep) { return (uint32_t)kstep * 2048; }
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -293,6 +300,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
         if (!mbar_wait(BAR(L::kKVFull), unit_iter & 1, wc)) { ok = false; break; }
         const uint32_t sK = base + L::kKOff, sV = base + L::kVOff;
+        const uint64_t dK = kmaj<kBlockN>(sK, 0), dV = kmaj<kBlockN>(sV, 0), dKmn = mnmaj<kBlockN>(sK, 0);
+        const uint64_t dDSmn = mnmaj<kBlockN>(base + L::kDSOff, 0);
         IterWin iw;  // walks forward only: the scan for the next iteration leads
         int a0 = 0;  // first computed iteration (n_it when the key tile is attended by none)
         while (a0 < bu.n_it && !bactive<D, SPARSE>(iw, p, bu, a0)) ++a0;
@@ -301,16 +310,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const uint32_t st = q_iter % L::kStages;
           if (!mbar_wait(BAR(L::kQFull + st), (q_iter / L::kStages) & 1, wc)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sQ = base + L::kQOff + st * L::kQT;
+          const uint64_t dQ = kmaj<BR>(base + L::kQOff + st * L::kQT, 0);
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks)
-            mma_ss(tmem + L::kColS, kmaj<kBlockN>(sK, ks), kmaj<BR>(sQ, ks), idesc_s, ks > 0);
+            mma_ss(tmem + L::kColS, sdesc_advance(dK, kmaj_off<kBlockN>(ks)), sdesc_advance(dQ, kmaj_off<BR>(ks)),
+                   idesc_s, ks > 0);
           tc_commit(BAR(L::kSFull));
         }
         for (int it = a0, nxt; it < bu.n_it; it = nxt) {  // active iterations only
           const uint32_t st = q_iter % L::kStages;
           const uint32_t sQ = base + L::kQOff + st * L::kQT;
           const uint32_t sDO = base + L::kDOOff + st * L::kQT;
+          const uint64_t dDO = kmaj<BR>(sDO, 0), dDOmn = mnmaj<BR>(sDO, 0), dQmn = mnmaj<BR>(sQ, 0);
           const uint32_t first = (it == a0);
           nxt = it + 1;
           while (nxt < bu.n_it && !bactive<D, SPARSE>(iw, p, bu, nxt)) ++nxt;
@@ -318,7 +329,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           // tile i-1, were consumed by dK(i-1), issued earlier)
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks)
-            mma_ss(tmem + L::kColDP, kmaj<kBlockN>(sV, ks), kmaj<BR>(sDO, ks), idesc_s, ks > 0);
+            mma_ss(tmem + L::kColDP, sdesc_advance(dV, kmaj_off<kBlockN>(ks)), sdesc_advance(dDO, kmaj_off<BR>(ks)),
+                   idesc_s, ks > 0);
           tc_commit(BAR(L::kDPFull));
           // dV += P^T dO_i
           if (!mbar_wait(BAR(L::kPFull), p_cnt & 1, wc)) { ok = false; break; }
@@ -327,16 +339,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < BR / 16; ++ks)
-            mma_ts(tmem + L::kColDV, tmem + L::kColS + L::packed_col(ks), mnmaj<BR>(sDO, ks), idesc_acc, (!first || ks > 0) ? 1u : 0u);
+            mma_ts(tmem + L::kColDV, tmem + L::kColS + L::packed_col(ks), sdesc_advance(dDOmn, mnmaj_off(ks)), idesc_acc,
+                   (!first || ks > 0) ? 1u : 0u);
           // S^T for the next query tile (the S region's P^T was consumed by dV above)
           if (nxt < bu.n_it) {
             const uint32_t st1 = (q_iter + 1) % L::kStages;
             if (!mbar_wait(BAR(L::kQFull + st1), ((q_iter + 1) / L::kStages) & 1, wc)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t sQ1 = base + L::kQOff + st1 * L::kQT;
+            const uint64_t dQ1 = kmaj<BR>(base + L::kQOff + st1 * L::kQT, 0);
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks)
-              mma_ss(tmem + L::kColS, kmaj<kBlockN>(sK, ks), kmaj<BR>(sQ1, ks), idesc_s, ks > 0);
+              mma_ss(tmem + L::kColS, sdesc_advance(dK, kmaj_off<kBlockN>(ks)), sdesc_advance(dQ1, kmaj_off<BR>(ks)),
+                     idesc_s, ks > 0);
             tc_commit(BAR(L::kSFull));
           }
           if (!mbar_wait(BAR(L::kDSFull), ds_cnt & 1, wc)) { ok = false; break; }
@@ -345,18 +359,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           // dK += dS^T Q_i
 #pragma unroll
           for (int ks = 0; ks < BR / 16; ++ks)
-            mma_ts(tmem + L::kColDK, tmem + L::kColDP + L::packed_col(ks), mnmaj<BR>(sQ, ks), idesc_acc,
+            mma_ts(tmem + L::kColDK, tmem + L::kColDP + L::packed_col(ks), sdesc_advance(dQmn, mnmaj_off(ks)), idesc_acc,
                    (!first || ks > 0) ? 1u : 0u);
           // dQ_i (d=64) or dQ_i^T (d=128) from dS^T in shared memory
           if (dq_cnt > 0 && !mbar_wait(BAR(L::kDQEmpty), (dq_cnt - 1) & 1, wc)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sDS = base + L::kDSOff;
 #pragma unroll
           for (int ks = 0; ks < kBlockN / 16; ++ks) {
-            if (D == 64)
-              mma_ss(tmem + L::kColDQ, mnmaj<kBlockN>(sDS, ks), mnmaj<kBlockN>(sK, ks), idesc_dq, ks > 0);
-            else
-              mma_ss(tmem + L::kColDQ, mnmaj<kBlockN>(sK, ks), mnmaj<kBlockN>(sDS, ks), idesc_dq, ks > 0);
+            const uint64_t a = sdesc_advance(D == 64 ? dDSmn : dKmn, mnmaj_off(ks));
+            const uint64_t b = sdesc_advance(D == 64 ? dKmn : dDSmn, mnmaj_off(ks));
+            mma_ss(tmem + L::kColDQ, a, b, idesc_dq, ks > 0);
           }
           tc_commit(BAR(L::kDQFull));
           ++dq_cnt;

@@ -43,9 +43,14 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only if max gr
 #ifndef FA_FWD_POLY_PAIR_MASK_D128
 #define FA_FWD_POLY_PAIR_MASK_D128 0x00
 #endif
-template <int D>
+// The FP8 variant's products take half the time of the 16-bit ones, so its
+// softmax is MUFU-bound at d = 128 as well.
+#ifndef FA_FWD_POLY_PAIR_MASK_FP8
+#define FA_FWD_POLY_PAIR_MASK_FP8 0x00
+#endif
+template <int D, bool FP8 = false>
 constexpr uint32_t poly_pair_mask() {
-  return D == 64 ? FA_FWD_POLY_PAIR_MASK_D64 : FA_FWD_POLY_PAIR_MASK_D128;
+  return FP8 ? FA_FWD_POLY_PAIR_MASK_FP8 : D == 64 ? FA_FWD_POLY_PAIR_MASK_D64 : FA_FWD_POLY_PAIR_MASK_D128;
 }
 // Register split.  Launch: 384 threads x 168 registers.  Warp w runs on SM
 // sub-partition w % 4, which therefore holds warps {k, k+4, k+8}: two softmax
@@ -98,8 +103,8 @@ struct UnitInfo {
   int nb_0, nb_1;  // key/value tiles each query tile may visit (0 = tile absent)
   int nmax;
   // Key/value tiles actually visited: the union of the two query tiles'
-  // active tiles (all of them when dense); each query tile visits those with
-  // index below its own nb, nbk_t of them.
+  // active tiles (all of them when dense), K of them; query tile t computes
+  // nbk_t of them (dense: its nb_t; block-sparse: the ones it attends).
   int K, nbk_0, nbk_1;
   __device__ __forceinline__ int r0(int t) const { return t ? r0_1 : r0_0; }
   __device__ __forceinline__ int nb(int t) const { return t ? nb_1 : nb_0; }
@@ -170,12 +175,9 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams& p) {
       w.seek(p, ui, j0);
       const uint32_t any = w.w0 | w.w1;
       // visited blocks below each tile's own nb
-      const int n0 = ui.nb_0 - j0, n1 = ui.nb_1 - j0;
-      const uint32_t lo0 = n0 >= 32 ? 0xffffffffu : (n0 > 0 ? (1u << n0) - 1u : 0u);
-      const uint32_t lo1 = n1 >= 32 ? 0xffffffffu : (n1 > 0 ? (1u << n1) - 1u : 0u);
       ui.K += __popc(any);
-      ui.nbk_0 += __popc(any & lo0);
-      ui.nbk_1 += __popc(any & lo1);
+      ui.nbk_0 += __popc(w.w0);    // blocks tile 0 attends (w0 is 0 past nb_0)
+      ui.nbk_1 += __popc(w.w1);
     }
   }
   return ui;
@@ -187,6 +189,10 @@ template <int D>
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kstep) {
   const uint32_t addr = tile + (uint32_t)(kstep >> 2) * (kBlockM * 128) + (uint32_t)(kstep & 3) * 32;
   return make_sdesc_sw128(addr, 16, 1024);
+}
+// Byte offset of K step `kstep` in such a tile (for sdesc_advance).
+__host__ __device__ constexpr uint32_t kmajor_off(int kstep) {
+  return (uint32_t)(kstep >> 2) * (kBlockM * 128) + (uint32_t)(kstep & 3) * 32;
 }
 
 // V tile as the MN-major B operand of O += P V: N = head dim (contiguous),
@@ -327,9 +333,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_fence_after();
         const uint32_t kv_base = kv_iter;
         if (ui.K == 0) tc_commit(BAR(L::kQEmpty + qb));  // no key block: Q is not read
+        // Block-sparse: each query tile computes only the visited blocks it
+        // attends (live); the other tile's blocks cost it no MMA and no
+        // softmax.  Dense: tile t is live at visited block j iff j < nb_t.
+        MaskWin mw;
+        int jb_cur = -1;                    // block index of visited block j
+        bool live_prev0 = false, live_prev1 = false, live_cur0 = false, live_cur1 = false;
+        int pv_done0 = 0, pv_done1 = 0;     // P V products issued per tile
         for (int j = 0; j <= ui.K && ok; ++j) {          // j counts visited blocks
           const uint32_t k_idx = kv_base + 2 * j, v_idx = kv_base + 2 * (j - 1) + 1;
           bool v_ready = false, k_ready = false;
+          if constexpr (SPARSE) {
+            live_prev0 = live_cur0;
+            live_prev1 = live_cur1;
+            live_cur0 = live_cur1 = false;
+            if (j < ui.K) {
+              do { ++jb_cur; } while (!unit_block<SPARSE>(p, ui, mw, jb_cur));
+              live_cur0 = mw.tile(0, jb_cur);
+              live_cur1 = mw.tile(1, jb_cur);
+            }
+          }
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
             const int nbt = ui.nbk(t);
@@ -338,11 +361,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const uint32_t colO = L::kColO0 + (uint32_t)D * t;
             const uint32_t pc = t ? p_cnt1 : p_cnt0;
             const uint32_t ou = t ? o_uses1 : o_uses0;
-            if (j >= 1 && j <= nbt) {
+            bool pv_now, s_now, first, last;
+            if constexpr (SPARSE) {
+              const int pvd = t ? pv_done1 : pv_done0;
+              pv_now = t ? live_prev1 : live_prev0;
+              s_now = t ? live_cur1 : live_cur0;
+              first = pvd == 0;
+              last = pvd + 1 == nbt;
+            } else {
+              pv_now = j >= 1 && j <= nbt;
+              s_now = j < nbt;
+              first = j == 1;
+              last = j == nbt;
+            }
+            if (pv_now) {
               // O_t (+)= P_t V_{j-1}
+              if constexpr (SPARSE) {
+                if (t) ++pv_done1; else ++pv_done0;
+              }
               ok = mbar_wait(BAR(L::kPFull + t), pc & 1, wc);
               if (t) ++p_cnt1; else ++p_cnt0;
-              if (ok && j == 1 && ou > 0) ok = mbar_wait(BAR(L::kOEmpty + t), (ou - 1) & 1, wc);
+              if (ok && first && ou > 0) ok = mbar_wait(BAR(L::kOEmpty + t), (ou - 1) & 1, wc);
               if (ok && !v_ready) {
                 ok = mbar_wait(BAR(L::kKVFull + v_idx % L::kSlots), (v_idx / L::kSlots) & 1, wc);
                 v_ready = true;
@@ -350,19 +389,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               if (!ok) continue;
               tc_fence_after();
               const uint32_t vt = base + L::kKVOff + (v_idx % L::kSlots) * L::kTile;
+              // descriptors built once per tile, stepped by constant offsets
               if constexpr (FP8) {
+                const uint64_t vd = kmajor_desc<128>(vt, 0);
 #pragma unroll
                 for (int ks = 0; ks < kBlockN / 32; ++ks)
-                  mma_ts_f8(tmem + colO, tmem + colS + 8u * ks, kmajor_desc<128>(vt, ks), idesc_pv,
-                            (j > 1 || ks > 0) ? 1u : 0u);
+                  mma_ts_f8(tmem + colO, tmem + colS + 8u * ks, sdesc_advance(vd, kmajor_off(ks)), idesc_pv,
+                            (!first || ks > 0) ? 1u : 0u);
               } else {
+                const uint64_t vd = v_desc(vt, 0);
 #pragma unroll
                 for (int ks = 0; ks < kBlockN / 16; ++ks)
-                  mma_ts(tmem + colO, tmem + colS + 8u * ks, v_desc(vt, ks), idesc_pv, (j > 1 || ks > 0) ? 1u : 0u);
+                  mma_ts(tmem + colO, tmem + colS + 8u * ks, sdesc_advance(vd, (uint32_t)ks * 2048), idesc_pv,
+                         (!first || ks > 0) ? 1u : 0u);
               }
-              if (j == nbt) tc_commit(BAR(L::kOFull + t));
+              if (last) tc_commit(BAR(L::kOFull + t));
             }
-            if (j < nbt) {
+            if (s_now) {
               // K_j is waited for only here, after the PV MMAs of block j-1
               // (which do not need it) have been issued.
               if (!k_ready) {
@@ -374,14 +417,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               // S_t = Q_t K_j^T
               const uint32_t qt = base + L::kQOff + (qb * 2 + t) * L::kTile;
               const uint32_t kt = base + L::kKVOff + (k_idx % L::kSlots) * L::kTile;
+              const uint64_t qd = kmajor_desc<D>(qt, 0), kd = kmajor_desc<D>(kt, 0);
               if constexpr (FP8) {
 #pragma unroll
                 for (int ks = 0; ks < D / 32; ++ks)
-                  mma_ss_f8(tmem + colS, kmajor_desc<D>(qt, ks), kmajor_desc<D>(kt, ks), idesc_s, ks > 0 ? 1u : 0u);
+                  mma_ss_f8(tmem + colS, sdesc_advance(qd, kmajor_off(ks)), sdesc_advance(kd, kmajor_off(ks)),
+                            idesc_s, ks > 0 ? 1u : 0u);
               } else {
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks)
-                  mma_ss(tmem + colS, kmajor_desc<D>(qt, ks), kmajor_desc<D>(kt, ks), idesc_s, ks > 0 ? 1u : 0u);
+                  mma_ss(tmem + colS, sdesc_advance(qd, kmajor_off(ks)), sdesc_advance(kd, kmajor_off(ks)), idesc_s,
+                         ks > 0 ? 1u : 0u);
               }
               tc_commit(BAR(L::kSFull + t));
             }
@@ -428,7 +474,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int jb = -1;                                 // index of the current key block
       MaskWin mw;
       for (int j = 0; j < nb; ++j) {
-        do { ++jb; } while (!unit_block<SPARSE>(p, ui, mw, jb));
+        if constexpr (SPARSE) {
+          do { ++jb; } while (!(unit_block<SPARSE>(p, ui, mw, jb) && mw.tile(t, jb)));
+        } else {
+          ++jb;
+        }
         ok = warp_all(mbar_wait(BAR(L::kSFull + t), s_cnt & 1, wc));
         if (!ok) break;
         ++s_cnt;
@@ -441,16 +491,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(sr[c]);
         const int kbase = jb * kBlockN;
-        // Block-sparse: a block visited for the other query tile only keeps
-        // nothing here.  Its scores are left as they are (finite: no causal or
-        // ragged mask is applied to it) and dropped below through the row
-        // max and the exponent, which is cheaper in registers than masking.
-        const bool dead = SPARSE && !mw.tile(t, jb);
         // factor from raw scores to log2 units (FP8: times both block scales)
         float c_l2 = sl2;
         if constexpr (FP8) c_l2 = sq_l2 * p.fp8_sk[(size_t)ui.kvbh * p.n_kv + jb];
-        if (dead) {
-        } else if (CAUSAL && jb == qblk) {
+        if (CAUSAL && jb == qblk) {
 #pragma unroll
           for (int c = 0; c < kBlockN; ++c)
             if (kbase + c > row) s[c] = -INFINITY;
@@ -468,7 +512,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int a = 0; a < 8; ++a) pm[a] = fmax3(pm[a], s[c + a], s[c + a + 8]);
         const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
-        const float m_new = fmaxf(m_run, dead ? -INFINITY : mx * c_l2);
+        const float m_new = fmaxf(m_run, mx * c_l2);
         // Until a row has seen a key, its O and l are zero: the first finite
         // max is taken as is, without a rescale.
         const bool fresh = m_run == -INFINITY;
@@ -497,18 +541,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
           }
         }
-        // -inf row: every P is 0.  Dead block: x = s * 0 - inf = -inf, P = 0.
-        const float neg_m = dead ? -INFINITY : (m_run == -INFINITY) ? 0.f : -m_run;
-        const float sl2x = dead ? 0.f : c_l2;
+        const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;  // -inf row: every P is 0
         float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int q = 0; q < kBlockN / 32; ++q) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float x0 = fmaf(s[32 * q + 2 * e], sl2x, neg_m);
-            const float x1 = fmaf(s[32 * q + 2 * e + 1], sl2x, neg_m);
-            const bool poly = (poly_pair_mask<D>() >> (e & 7)) & 1u;
+            const float x0 = fmaf(s[32 * q + 2 * e], c_l2, neg_m);
+            const float x1 = fmaf(s[32 * q + 2 * e + 1], c_l2, neg_m);
+            const bool poly = (poly_pair_mask<D, FP8>() >> (e & 7)) & 1u;
             const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
             const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
             ps[e & 3] += p0 + p1;

@@ -236,6 +236,15 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr, uint32_t lb
   return d;
 }
 
+// The descriptor of the same operand `bytes` further on in shared memory (a
+// K step inside a swizzle atom, or the next column block).  The address field
+// (bits 0-13, address >> 4) does not overflow for addresses below 256 KB, so
+// one add replaces rebuilding the descriptor in the MMA issuer's hot loop.
+__device__ __forceinline__ uint64_t sdesc_advance(uint64_t d, uint32_t bytes) {
+  const uint32_t lo = (uint32_t)d + (bytes >> 4);
+  return ((d >> 32) << 32) | lo;
+}
+
 // Tensor-memory loads/stores, 32 lanes x 32 bits, repeated N times: thread i
 // of the warp reads/writes lane (warp quadrant * 32 + i), N consecutive columns.
 #define FA_TMEM_LD_X16(taddr, r)                                                                  \

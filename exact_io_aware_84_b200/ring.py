@@ -37,7 +37,7 @@ from __future__ import annotations
 
 from typing import List, Optional, Sequence, Tuple
 
-__all__ = ["ring_schedule", "RingComm", "CudaChunkOps", "ring_attention_fwd", "ring_attention_bwd"]
+__all__ = ["ring_schedule", "RingComm", "ThreadRing", "CudaChunkOps", "ring_attention_fwd", "ring_attention_bwd"]
 
 
 def ring_schedule(rank: int, world: int, causal: bool) -> List[Tuple[int, int, bool, bool]]:
@@ -85,6 +85,68 @@ class RingComm:
     def wait(handles):
         for h in handles or ():
             h.wait()
+
+
+class ThreadRing:
+    """A ring of ``world`` ranks emulated by host threads of one process on
+    one device (one thread per rank, all launching on the same stream).
+    ``comm(rank)`` gives rank ``rank`` its end: ``exchange`` posts the
+    tensors to send, waits for every rank at a barrier, copies the
+    predecessor's tensors into the receive buffers (device copies on the
+    shared stream, so they run after the kernels that produced them) and
+    meets the others at a second barrier before anyone may overwrite what it
+    posted.  The device never waits on anything: the ranks' kernels run one
+    after another."""
+
+    def __init__(self, world: int, timeout: float = 120.0):
+        import threading
+
+        self.world = world
+        self.slots = [None] * world
+        self.barrier = threading.Barrier(world, timeout=timeout)
+
+    def comm(self, rank: int):
+        return _ThreadComm(self, rank)
+
+    def run(self, fn):
+        """Run ``fn(rank)`` for every rank on its own thread; re-raise the
+        first error (breaking the barrier, so that the other ranks stop)."""
+        import threading
+
+        errs = []
+
+        def body(r):
+            try:
+                fn(r)
+            except BaseException as e:  # noqa: BLE001 - re-raised below
+                errs.append(e)
+                self.barrier.abort()
+
+        threads = [threading.Thread(target=body, args=(r,)) for r in range(self.world)]
+        for t in threads:
+            t.start()
+        for t in threads:
+            t.join()
+        if errs:
+            raise errs[0]
+
+
+class _ThreadComm:
+    def __init__(self, ring: ThreadRing, rank: int):
+        self.ring, self.rank, self.world = ring, rank, ring.world
+
+    def exchange(self, send: Sequence, recv: Sequence):
+        ring = self.ring
+        ring.slots[self.rank] = list(send)
+        ring.barrier.wait()
+        for r, s in zip(recv, ring.slots[(self.rank - 1) % self.world]):
+            r.copy_(s)
+        ring.barrier.wait()
+        return None
+
+    @staticmethod
+    def wait(handles):
+        pass
 
 
 class CudaChunkOps:

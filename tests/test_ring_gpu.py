@@ -9,14 +9,12 @@
   barrier.  The concatenated results must match the oracle's full attention.
 """
 
-import threading
-
 import numpy as np
 import pytest
 import torch
 
 import exact_io_aware_84_b200 as fa
-from exact_io_aware_84_b200.ring import ring_attention_bwd, ring_attention_fwd
+from exact_io_aware_84_b200.ring import ThreadRing, ring_attention_bwd, ring_attention_fwd
 from oracle import attn_bwd_ref, attn_fwd_ref, merge_partials_ref
 from parity import check_grads, check_o_lse, to64
 
@@ -59,34 +57,6 @@ def test_accumulate_and_convert(dtype, n):
     assert torch.equal(out.cpu(), want.to(dtype))   # round to nearest even
 
 
-class _Shared:
-    def __init__(self, world):
-        self.world = world
-        self.slots = [None] * world
-        self.barrier = threading.Barrier(world, timeout=120)
-
-
-class _LocalComm:
-    """In-process ring exchange: every rank posts its tensors, then copies its
-    predecessor's into its receive buffers (on the shared CUDA stream, so the
-    copy runs after the kernels that produced them)."""
-
-    def __init__(self, shared, rank):
-        self.sh, self.rank, self.world = shared, rank, shared.world
-
-    def exchange(self, send, recv):
-        self.sh.slots[self.rank] = list(send)
-        self.sh.barrier.wait()
-        for r, s in zip(recv, self.sh.slots[(self.rank - 1) % self.world]):
-            r.copy_(s)
-        self.sh.barrier.wait()
-        return None
-
-    @staticmethod
-    def wait(handles):
-        pass
-
-
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("world,n,d", [(2, 384, 64), (4, 300, 128), (3, 1000, 64)])
 def test_ring_emulated_on_one_gpu_matches_full_attention(world, n, d, causal):
@@ -94,29 +64,19 @@ def test_ring_emulated_on_one_gpu_matches_full_attention(world, n, d, causal):
     g = torch.Generator().manual_seed(world * 100 + n + d)
     q, k, v, do = (torch.randn(B, H, world * n, d, generator=g).to(torch.bfloat16) for _ in range(4))
     scale = d ** -0.5
-    sh = _Shared(world)
-    res, errs = [None] * world, []
+    ring = ThreadRing(world)
+    res = [None] * world
 
     def run(r):
-        try:
-            sl = slice(r * n, (r + 1) * n)
-            lq, lk, lv, ldo = (x[:, :, sl].contiguous().cuda() for x in (q, k, v, do))
-            comm = _LocalComm(sh, r)
-            o, lse, o32 = ring_attention_fwd(lq, lk, lv, scale=scale, causal=causal, comm=comm)
-            grads = ring_attention_bwd(lq, lk, lv, o32, ldo, lse, scale=scale, causal=causal, comm=comm)
-            torch.cuda.synchronize()
-            res[r] = (o, lse) + tuple(grads)
-        except BaseException as e:  # noqa: BLE001 - reported below
-            errs.append(e)
-            sh.barrier.abort()
+        sl = slice(r * n, (r + 1) * n)
+        lq, lk, lv, ldo = (x[:, :, sl].contiguous().cuda() for x in (q, k, v, do))
+        comm = ring.comm(r)
+        o, lse, o32 = ring_attention_fwd(lq, lk, lv, scale=scale, causal=causal, comm=comm)
+        grads = ring_attention_bwd(lq, lk, lv, o32, ldo, lse, scale=scale, causal=causal, comm=comm)
+        torch.cuda.synchronize()
+        res[r] = (o, lse) + tuple(grads)
 
-    threads = [threading.Thread(target=run, args=(r,)) for r in range(world)]
-    for t in threads:
-        t.start()
-    for t in threads:
-        t.join()
-    if errs:
-        raise errs[0]
+    ring.run(run)
     assert fa.fa_last_device_status() == fa.FA_OK
     cat = lambda i: torch.cat([res[r][i] for r in range(world)], dim=-2 if i != 1 else -1)
     o_ref, lse_ref = attn_fwd_ref(to64(q), to64(k), to64(v), scale, causal)

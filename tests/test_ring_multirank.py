@@ -116,3 +116,46 @@ def test_ring_schedule_covers_every_pair_once(world):
 def test_ring_schedule_rejects_bad_rank():
     with pytest.raises(ValueError):
         ring_schedule(3, 3, False)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_thread_ring_equals_full_attention(causal):
+    # the in-process ring (one host thread per rank) with the oracle as the
+    # chunk steps, on CPU tensors
+    from oracle import attn_bwd_ref, attn_fwd_ref
+
+    from exact_io_aware_84_b200.ring import ThreadRing, ring_attention_bwd, ring_attention_fwd
+    world, n = 4, 3
+    q, k, v, do = _full_inputs(world, n, causal)
+    ring = ThreadRing(world)
+    out = [None] * world
+
+    def run(r):
+        sl = slice(r * n, (r + 1) * n)
+        lq, lk, lv, ldo = (x[:, :, sl].contiguous() for x in (q, k, v, do))
+        comm = ring.comm(r)
+        o, lse, o32 = ring_attention_fwd(lq, lk, lv, scale=0.6, causal=causal, ops=OracleOps(), comm=comm)
+        out[r] = (o, lse) + ring_attention_bwd(lq, lk, lv, o32, ldo, lse, scale=0.6, causal=causal,
+                                               ops=OracleOps(), comm=comm)
+
+    ring.run(run)
+    o_ref, lse_ref = attn_fwd_ref(q.numpy(), k.numpy(), v.numpy(), 0.6, causal)
+    grads = attn_bwd_ref(q.numpy(), k.numpy(), v.numpy(), do.numpy(), 0.6, causal)
+    cat = lambda i, ax: np.concatenate([out[r][i].numpy() for r in range(world)], axis=ax)
+    np.testing.assert_allclose(cat(0, -2), o_ref, atol=1e-12)
+    np.testing.assert_allclose(cat(1, -1), lse_ref, atol=1e-12)
+    for i, ref in zip((2, 3, 4), grads):
+        np.testing.assert_allclose(cat(i, -2), ref, atol=1e-12)
+
+
+def test_thread_ring_reraises_a_rank_error():
+    from exact_io_aware_84_b200.ring import ThreadRing
+    ring = ThreadRing(3, timeout=10)
+
+    def run(r):
+        if r == 1:
+            raise RuntimeError("rank 1 failed")
+        ring.comm(r).exchange([torch.zeros(2)], [torch.zeros(2)])
+
+    with pytest.raises(RuntimeError, match="rank 1 failed"):
+        ring.run(run)
