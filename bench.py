@@ -553,16 +553,43 @@ def _e2e(fa, torch, w, x, dev, stream, flops, world, args):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
+def _code_only(text):
+    """C/C++/CUDA source without comments and blank lines (what the compiler
+    sees; comment edits do not change the kernels)."""
+    import re
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"' or c == "'":          # string or character literal
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = [ln.rstrip() for ln in "".join(out).split("\n")]
+    return "\n".join(ln for ln in lines if ln.strip())
+
+
 def kernel_sources_hash():
-    """sha1 prefix of the CUDA sources (file names and contents, sorted)."""
+    """sha1 prefix of the CUDA sources' code (file names and contents without
+    comments, sorted)."""
     import glob
     import hashlib
     h = hashlib.sha1()
     for f in sorted(glob.glob(os.path.join(ROOT, "exact_io_aware_84_b200", "csrc", "*"))):
         if f.endswith((".cu", ".cuh", ".h")):
             h.update(os.path.basename(f).encode())
-            with open(f, "rb") as fh:
-                h.update(fh.read())
+            with open(f, encoding="utf-8") as fh:
+                h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -14,16 +14,18 @@
 //
 // fa_bwd_main works transposed (keys on the 128 tensor-memory lanes):
 //   S^T = K_j Q_i^T, dP^T = V_j dO_i^T            (SS MMAs, M = 128 keys)
-//   P^T = exp2(S^T * scale*log2e - LSE_i*log2e)    (softmax warpgroup)
-//   dS^T = P^T o (dP^T - D_i)                      (softmax warpgroup)
+//   P^T = exp2(S^T * scale*log2e - LSE_i*log2e)    (compute warpgroups)
+//   dS^T = P^T o (dP^T - D_i)                      (compute warpgroups)
 //   dV += P^T dO_i, dK += dS^T Q_i                 (TS MMAs, A from TMEM)
 //   d = 64 : dQ_i   = dS K_j      (M = 128 queries, both operands MN-major)
 //   d = 128: dQ_i^T = K_j^T dS^T  (M = 128 head dims, both operands MN-major)
 // Query tile BR = 128 rows for d = 64 and 64 rows for d = 128, so that
 // S^T | dP^T | dV | dK | dQ fit in the 512 tensor-memory columns (448 used).
 // Roles (384 threads):
-//   warps 0-3   softmax warpgroup (thread = key = TMEM lane)
-//   warps 4-7   dQ / dK / dV epilogue warpgroup
+//   warps 0-7   two compute warpgroups (thread = key = TMEM lane), each owning
+//               half of every query tile's columns: P^T, the staging of the
+//               previous tile's dQ, dS^T; at the end of a unit each writes
+//               half of the head dims of dK and dV
 //   warp  8     TMA producer      warp 9   MMA issuer      warps 10-11 idle
 #include <cuda_fp16.h>
 
