@@ -297,15 +297,34 @@ def run_native(args):
         # the sequence split into R chunks, one per emulated rank; every rank
         # runs the ring forward, then the ring backward (merges, fp32
         # accumulation and conversions included); same FLOPs as full attention
-        from exact_io_aware_84_b200.ring import ThreadRing, ring_attention_bwd, ring_attention_fwd
+        from exact_io_aware_84_b200.ring import RingComm, ThreadRing, ring_attention_bwd, ring_attention_fwd
+        if world > 1:
+            # one rank per GPU, each holding the workload's sequence as its
+            # chunk (the ring's sequence is world x N; per-GPU work grows with
+            # the world, as each rank attends to every chunk): NCCL
+            # point-to-point over NVLink between neighbouring ranks
+            comm = RingComm()
+            f_fwd = attn_fwd_flops(B, H, world * N, d, w.causal) / world
+            variant.update(ring_size=world, chunk=N, transfers="NCCL point-to-point between GPUs")
+            ring_state = {}
+
+            def step():
+                ring_state["f"] = ring_attention_fwd(g["q"], g["k"], g["v"], scale=w.scale, causal=w.causal, comm=comm)
+                ev_mid.record(stream)
+                if w.backward:
+                    _, l_r, o32_r = ring_state["f"]
+                    ring_attention_bwd(g["q"], g["k"], g["v"], o32_r, g["do"], l_r, scale=w.scale, causal=w.causal,
+                                       comm=comm)
         R = args.ring_size
-        if N % R:
+        if world == 1 and N % R:
             raise SystemExit(f"N = {N} is not a multiple of the ring size {R}")
         n = N // R
-        chunks = [{k: t[:, :, r * n:(r + 1) * n].contiguous() for k, t in g.items()} for r in range(R)]
+        chunks = [{k: t[:, :, r * n:(r + 1) * n].contiguous() for k, t in g.items()} for r in range(R)] \
+            if world == 1 else []
         ring = ThreadRing(R)
         state = [None] * R
-        variant.update(ring_size=R, chunk=n, transfers="device copies on one GPU (no NVLink)")
+        if world == 1:
+            variant.update(ring_size=R, chunk=n, transfers="device copies on one GPU (no NVLink)")
 
         def fwd_rank(r):
             torch.cuda.set_device(dev)
@@ -320,11 +339,12 @@ def run_native(args):
             ring_attention_bwd(c["q"], c["k"], c["v"], o32_r, c["do"], l_r, scale=w.scale, causal=w.causal,
                                comm=ring.comm(r))
 
-        def step():
-            ring.run(fwd_rank)
-            ev_mid.record(stream)
-            if w.backward:
-                ring.run(bwd_rank)
+        if world == 1:
+            def step():
+                ring.run(fwd_rank)
+                ev_mid.record(stream)
+                if w.backward:
+                    ring.run(bwd_rank)
     else:
         # block-sparse: per head, each 128x128 tile kept with probability 1/2
         # (seeded); FLOPs count only the (query, key) pairs actually attended
@@ -350,10 +370,14 @@ def run_native(args):
     launches_per_step = (4 if args.variant == "fp8" else 1) + (3 if with_bwd else 0)
     if args.variant == "ring":
         # per rank and step: forward 1 (+1 merge), backward 3 + 3 accumulates;
-        # per rank: 1 + 3 conversions (skipped chunk pairs launch nothing)
-        R = args.ring_size
+        # per rank: 1 + 3 conversions (skipped chunk pairs launch nothing);
+        # counted for all emulated ranks on one GPU, for this rank with NCCL
+        R = args.ring_size if world == 1 else world
         pairs = R * (R + 1) // 2 if w.causal else R * R
         launches_per_step = (pairs + (pairs - R) + R) + ((6 * pairs + 3 * R) if with_bwd else 0)
+        if world > 1:  # this rank's own launches (rank 0 prints)
+            pr = rank + 1 if w.causal else world
+            launches_per_step = (2 * pr) + ((6 * pr + 3) if with_bwd else 0)
     f_bwd = 2.5 * f_fwd if with_bwd else 0.0
     flops = f_fwd + f_bwd
 

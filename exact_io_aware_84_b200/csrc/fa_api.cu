@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <atomic>
 #include <cstdint>
@@ -14,6 +15,15 @@
 #include "sm100_ptx.cuh"
 
 namespace fa {
+
+// Host-side NVTX range around each entry point (visible in timeline
+// profilers; a no-op when none is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Device status word: 0 = OK, else the fa_status of a kernel that gave up.
 __device__ int g_device_status = 0;
@@ -247,11 +257,13 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
            float scale, int causal, int dtype, void* stream) {
+  NvtxRange nvtx_range("fa_fwd");
   return fwd_impl(q, k, v, o, lse, B, H, H, N, d, scale, causal, dtype, stream);
 }
 
 int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
                int d, float scale, int causal, int dtype, void* stream) {
+  NvtxRange nvtx_range("fa_fwd_gqa");
   return fwd_impl(q, k, v, o, lse, B, H, Hkv, N, d, scale, causal, dtype, stream);
 }
 
@@ -322,6 +334,7 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
            void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
            float scale, int causal, int dtype, void* stream) {
+  NvtxRange nvtx_range("fa_bwd");
   return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, H, N, d, scale, causal,
                   dtype, stream);
 }
@@ -329,6 +342,7 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
 int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int N,
                int d, float scale, int causal, int dtype, void* stream) {
+  NvtxRange nvtx_range("fa_bwd_gqa");
   return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, N, d, scale, causal,
                   dtype, stream);
 }
@@ -336,6 +350,7 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const
 int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
                        const unsigned char* block_mask, long long mask_head_stride, int B, int H, int N, int d,
                        float scale, int causal, int dtype, void* stream) {
+  NvtxRange nvtx_range("fa_fwd_blocksparse");
   if (!block_mask) return FA_ERR_INVALID_ARG;
   return fwd_impl(q, k, v, o, lse, B, H, H, N, d, scale, causal, dtype, stream, block_mask, mask_head_stride);
 }
@@ -344,6 +359,7 @@ int fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* 
                        const float* lse, const unsigned char* block_mask, long long mask_head_stride, void* dq,
                        void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
                        float scale, int causal, int dtype, void* stream) {
+  NvtxRange nvtx_range("fa_bwd_blocksparse");
   if (!block_mask) return FA_ERR_INVALID_ARG;
   return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, H, N, d, scale, causal,
                   dtype, stream, block_mask, mask_head_stride);
@@ -372,12 +388,14 @@ static int fp8_prep(const void* q, const void* k, const void* v, const float* si
 
 int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* signs, void* workspace,
                     size_t workspace_bytes, int B, int H, int N, int d, int dtype, void* stream) {
+  NvtxRange nvtx_range("fa_fp8_quantize");
   return fp8_prep(q, k, v, signs, workspace, workspace_bytes, B, H, N, d, dtype, stream);
 }
 
 int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, const float* signs,
                void* workspace, size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
                int dtype, void* stream) {
+  NvtxRange nvtx_range("fa_fwd_fp8");
   if (!o || !lse) return FA_ERR_INVALID_ARG;
   int st = check_common(B, H, N, d, scale, dtype);
   if (st != FA_OK) return st;
@@ -418,6 +436,7 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
 
 int fa_merge(float* o, float* lse, const float* o_part, const float* lse_part, void* out, int out_dtype,
              long long rows, int d, void* stream) {
+  NvtxRange nvtx_range("fa_merge");
   if (rows < 0) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (out_dtype < -1 || out_dtype > FA_FP16) return FA_ERR_UNSUPPORTED;
@@ -436,6 +455,7 @@ int fa_merge(float* o, float* lse, const float* o_part, const float* lse_part, v
 }
 
 int fa_grad_accumulate(float* acc, const void* src, long long n, int src_dtype, void* stream) {
+  NvtxRange nvtx_range("fa_grad_accumulate");
   if (n < 0) return FA_ERR_INVALID_ARG;
   if (src_dtype != FA_BF16 && src_dtype != FA_FP16) return FA_ERR_UNSUPPORTED;
   if (n == 0) return FA_OK;
@@ -449,6 +469,7 @@ int fa_grad_accumulate(float* acc, const void* src, long long n, int src_dtype, 
 }
 
 int fa_convert(void* dst, const float* src, long long n, int dst_dtype, void* stream) {
+  NvtxRange nvtx_range("fa_convert");
   if (n < 0) return FA_ERR_INVALID_ARG;
   if (dst_dtype != FA_BF16 && dst_dtype != FA_FP16) return FA_ERR_UNSUPPORTED;
   if (n == 0) return FA_OK;

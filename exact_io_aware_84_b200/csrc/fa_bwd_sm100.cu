@@ -621,70 +621,77 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
-// D_i = sum_c dO_ic O_ic; lse2_i = LSE_i * log2(e); both +0 / +inf on the
-// padding rows N..n_pad-1; dQacc rows zeroed.  One warp per row.  O is read
-// as 16-bit, or as fp32 for the O32 storage codes.
+// D_i = sum_c dO_ic O_ic and LSE_i * log2(e) per row (+inf on the padding
+// rows N..n_pad-1 and on rows with LSE = -inf), and the rows of dQacc zeroed.
+// D / 8 lanes per row, 8 elements (16 bytes of 16-bit data) per lane, so a
+// warp covers 32 / (D / 8) rows per pass with 16-byte accesses; warps stride
+// over the row groups.  O is read as 16-bit, or as fp32 for the O32 codes.
 template <int D, bool BF16, bool O32>
 __global__ void __launch_bounds__(256) fa_bwd_prep(const BwdParams p) {
-  const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  constexpr int L = D / 8;            // lanes per row
+  constexpr int RPW = 32 / L;         // rows per warp pass
   const int lane = threadIdx.x & 31;
-  const int total = p.bh * p.n_pad;
-  if (warp_global >= total) return;
-  const int bh = warp_global / p.n_pad;
-  const int row = warp_global % p.n_pad;
-  constexpr int PER = D / 32;  // elements per lane (2 or 4)
-  float acc = 0.f;
-  if (row < p.N) {
-    const size_t off = ((size_t)bh * p.N + row) * D + (size_t)lane * PER;
-    const uint32_t* d32 = reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(p.dout) + off * 2);
-    float ov[PER], dv[PER];
+  const int sub = lane % L, rsub = lane / L;
+  const long long groups = ((long long)p.bh * p.n_pad + RPW - 1) / RPW;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long g = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); g < groups; g += warps) {
+    const long long prow = g * RPW + rsub;           // bh * n_pad + row
+    const bool valid = prow < (long long)p.bh * p.n_pad;
+    const int bh = valid ? (int)(prow / p.n_pad) : 0;
+    const int row = valid ? (int)(prow % p.n_pad) : p.n_pad;
+    float acc = 0.f;
+    if (valid && row < p.N) {
+      const size_t off = ((size_t)bh * p.N + row) * D + (size_t)sub * 8;
+      const uint4 dw = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.dout) + off * 2);
+      float dv[8], ov[8];
+      const uint32_t dws[4] = {dw.x, dw.y, dw.z, dw.w};
 #pragma unroll
-    for (int e = 0; e < PER / 2; ++e) {
-      const uint32_t w = d32[e];
-      if constexpr (BF16) {
-        dv[2 * e] = __uint_as_float(w << 16);
-        dv[2 * e + 1] = __uint_as_float(w & 0xFFFF0000u);
-      } else {
-        const __half2 h = *reinterpret_cast<const __half2*>(&w);
-        dv[2 * e] = __low2float(h);
-        dv[2 * e + 1] = __high2float(h);
-      }
-    }
-    if constexpr (O32) {
-      const float* o32p = reinterpret_cast<const float*>(p.o) + off;
-#pragma unroll
-      for (int e = 0; e < PER; ++e) ov[e] = o32p[e];
-    } else {
-      const uint32_t* o16 = reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(p.o) + off * 2);
-#pragma unroll
-      for (int e = 0; e < PER / 2; ++e) {
-        const uint32_t w = o16[e];
+      for (int e = 0; e < 4; ++e) {
         if constexpr (BF16) {
-          ov[2 * e] = __uint_as_float(w << 16);
-          ov[2 * e + 1] = __uint_as_float(w & 0xFFFF0000u);
+          dv[2 * e] = __uint_as_float(dws[e] << 16);
+          dv[2 * e + 1] = __uint_as_float(dws[e] & 0xFFFF0000u);
         } else {
-          const __half2 h = *reinterpret_cast<const __half2*>(&w);
-          ov[2 * e] = __low2float(h);
-          ov[2 * e + 1] = __high2float(h);
+          dv[2 * e] = __half2float(__ushort_as_half((unsigned short)(dws[e] & 0xFFFFu)));
+          dv[2 * e + 1] = __half2float(__ushort_as_half((unsigned short)(dws[e] >> 16)));
         }
       }
+      if constexpr (O32) {
+        const float4* o4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.o) + off);
+        const float4 a = o4[0], b = o4[1];
+        ov[0] = a.x; ov[1] = a.y; ov[2] = a.z; ov[3] = a.w;
+        ov[4] = b.x; ov[5] = b.y; ov[6] = b.z; ov[7] = b.w;
+      } else {
+        const uint4 ow = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.o) + off * 2);
+        const uint32_t ows[4] = {ow.x, ow.y, ow.z, ow.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if constexpr (BF16) {
+            ov[2 * e] = __uint_as_float(ows[e] << 16);
+            ov[2 * e + 1] = __uint_as_float(ows[e] & 0xFFFF0000u);
+          } else {
+            ov[2 * e] = __half2float(__ushort_as_half((unsigned short)(ows[e] & 0xFFFFu)));
+            ov[2 * e + 1] = __half2float(__ushort_as_half((unsigned short)(ows[e] >> 16)));
+          }
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc = fmaf(ov[e], dv[e], acc);
     }
 #pragma unroll
-    for (int e = 0; e < PER; ++e) acc = fmaf(ov[e], dv[e], acc);
+    for (int s = L / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    if (valid) {
+      if (sub == 0) {
+        p.dvec[prow] = acc;
+        // padding rows and rows with no kept key (LSE = -inf, block-sparse)
+        // get +inf, so that any P recomputed for them is 0
+        const float l = row < p.N ? p.lse[(size_t)bh * p.N + row] : -INFINITY;
+        p.lse2[prow] = l > -INFINITY ? l * 1.4426950408889634f : INFINITY;
+      }
+      float4* acc_row = reinterpret_cast<float4*>(p.dq_acc + prow * D) + 2 * sub;
+      acc_row[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      acc_row[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
-#pragma unroll
-  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  const size_t prow = (size_t)bh * p.n_pad + row;
-  if (lane == 0) {
-    p.dvec[prow] = acc;
-    // padding rows and rows with no kept key (LSE = -inf, block-sparse) get
-    // +inf, so that any P recomputed for them is 0
-    const float l = row < p.N ? p.lse[(size_t)bh * p.N + row] : -INFINITY;
-    p.lse2[prow] = l > -INFINITY ? l * 1.4426950408889634f : INFINITY;
-  }
-  float4* acc_row = reinterpret_cast<float4*>(p.dq_acc + prow * D);
-#pragma unroll
-  for (int e = lane; e < D / 4; e += 32) acc_row[e] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // dQ = dtype(dQacc) for the real rows.  One thread per 8 elements.
@@ -706,8 +713,11 @@ template <int D, bool BF16, bool CAUSAL>
 cudaError_t launch_bwd_t(bool o32, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& tdo, const BwdParams& p, int grid, cudaStream_t st) {
   {
-    const long long warps = (long long)p.bh * p.n_pad;
-    const int blocks = (int)((warps * 32 + 255) / 256);
+    // row groups of 32 / (D / 8) rows per warp; a grid of up to 16 blocks of
+    // 8 warps per SM strides over them
+    const long long groups = ((long long)p.bh * p.n_pad + 32 / (D / 8) - 1) / (32 / (D / 8));
+    const long long want = (groups + 7) / 8;
+    const int blocks = (int)(want < 148LL * 16 ? want : 148LL * 16);
     if (o32)
       fa_bwd_prep<D, BF16, true><<<blocks, 256, 0, st>>>(p);
     else
