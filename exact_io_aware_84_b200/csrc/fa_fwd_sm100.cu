@@ -85,7 +85,10 @@ struct FwdLayout {
   static constexpr int kPFull = kSFull + 2;      // [2]
   static constexpr int kOFull = kPFull + 2;      // [2]
   static constexpr int kOEmpty = kOFull + 2;     // [2]
-  static constexpr int kDrain = kOEmpty + 2;
+  // Separate P (d = 64, 16-bit): S read by the softmax / P V product done
+  static constexpr int kSFree = kOEmpty + 2;     // [2]
+  static constexpr int kPVDone = kSFree + 2;     // [2]
+  static constexpr int kDrain = kPVDone + 2;
   static constexpr int kNumBars = kDrain + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
@@ -93,6 +96,7 @@ struct FwdLayout {
   // tensor-memory columns
   static constexpr uint32_t kColS0 = 0;
   static constexpr uint32_t kColO0 = 256;
+  static constexpr uint32_t kColP0 = 384;  // separate P (d = 64): P_0 | P_1, 64 columns each
   static_assert(kAlloc <= 232448, "shared memory overflow");
 };
 
@@ -211,13 +215,22 @@ __device__ __forceinline__ uint64_t v_desc(uint32_t tile, int kstep) {
 // dimension, 128 keys); the epilogue applies V's per-channel scales.  The
 // running sum l adds the unrounded P.  P stays within [0, 2^8] (the stale
 // max is at most 2^8 below the true one), inside e4m3's range of 448.
-template <int D, bool BF16, bool O32, bool CAUSAL, bool SPARSE, bool FP8 = false>
+template <int D, bool BF16, bool O32, bool CAUSAL, bool SPARSE, bool FP8 = false, bool SEPP = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   static_assert(!FP8 || (D == 128 && !SPARSE), "the FP8 variant is dense, head dim 128");
   using L = FwdLayout<D, FP8>;
   constexpr int kQKBoxes = FP8 ? 1 : D / 64;   // 128-byte column blocks per Q / K tile
+  // SEPP (d = 64 leaves 128 tensor-memory columns free): each tile's P gets
+  // its own region, so S_t(j+1) can be issued as soon as the softmax has read
+  // S_t(j) (instead of after P_t(j) has been consumed) and each tile's
+  // softmax runs block after block; the two tiles' softmaxes overlap.  The
+  // softmax waits for the previous P V product before it rescales O or
+  // overwrites P.  This shortens the per-block chain (a gain for short
+  // sequences, whose units are a few blocks long) but makes the softmaxes
+  // share the MUFU (a loss on long sequences); the launcher chooses.
+  constexpr bool kSepP = SEPP && (D == 64) && !FP8 && !SPARSE;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -243,6 +256,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(BAR(L::kPFull + t), 128);
       mbar_init(BAR(L::kOFull + t), 1);
       mbar_init(BAR(L::kOEmpty + t), 128);
+      mbar_init(BAR(L::kSFree + t), 128);
+      mbar_init(BAR(L::kPVDone + t), 1);
     }
     mbar_init(BAR(L::kDrain), 1);
     *abort_flag = 0;
@@ -325,6 +340,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       constexpr uint32_t idesc_pv = make_idesc_f16(FP8 ? false : BF16, kBlockM, D, false, !FP8);
       uint32_t kv_iter = 0, unit_iter = 0;
       uint32_t p_cnt0 = 0, p_cnt1 = 0, o_uses0 = 0, o_uses1 = 0;
+      uint32_t s_iss0 = 0, s_iss1 = 0;   // S MMAs issued per tile (separate-P pipeline)
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
         const UnitInfo ui = decode_unit<CAUSAL, SPARSE>(u, p);
@@ -333,6 +349,67 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_fence_after();
         const uint32_t kv_base = kv_iter;
         if (ui.K == 0) tc_commit(BAR(L::kQEmpty + qb));  // no key block: Q is not read
+        if constexpr (kSepP) {
+          // Per visited block j: first S_t(j) for both tiles (each after the
+          // softmax has read S_t(j-1)), then P_t(j-1) V_{j-1}.
+          for (int j = 0; j <= ui.K && ok; ++j) {
+            const uint32_t k_idx = kv_base + 2 * j, v_idx = kv_base + 2 * (j - 1) + 1;
+            bool k_ready = false, v_ready = false;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (!ok || j >= ui.nb(t)) continue;
+              uint32_t& sc = t ? s_iss1 : s_iss0;
+              if (sc > 0) ok = mbar_wait(BAR(L::kSFree + t), (sc - 1) & 1, wc);
+              if (ok && !k_ready) {
+                ok = mbar_wait(BAR(L::kKVFull + k_idx % L::kSlots), (k_idx / L::kSlots) & 1, wc);
+                k_ready = true;
+              }
+              if (!ok) continue;
+              tc_fence_after();
+              const uint32_t qt = base + L::kQOff + (qb * 2 + t) * L::kTile;
+              const uint32_t kt = base + L::kKVOff + (k_idx % L::kSlots) * L::kTile;
+              const uint64_t qd = kmajor_desc<D>(qt, 0), kd = kmajor_desc<D>(kt, 0);
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks)
+                mma_ss(tmem + L::kColS0 + 128u * t, sdesc_advance(qd, kmajor_off(ks)), sdesc_advance(kd, kmajor_off(ks)),
+                       idesc_s, ks > 0 ? 1u : 0u);
+              tc_commit(BAR(L::kSFull + t));
+              ++sc;
+            }
+            if (!ok) break;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              const int nbt = ui.nb(t);
+              if (!ok || j < 1 || j > nbt) continue;
+              const uint32_t pc = t ? p_cnt1 : p_cnt0;
+              const uint32_t ou = t ? o_uses1 : o_uses0;
+              ok = mbar_wait(BAR(L::kPFull + t), pc & 1, wc);
+              if (t) ++p_cnt1; else ++p_cnt0;
+              if (ok && j == 1 && ou > 0) ok = mbar_wait(BAR(L::kOEmpty + t), (ou - 1) & 1, wc);
+              if (ok && !v_ready) {
+                ok = mbar_wait(BAR(L::kKVFull + v_idx % L::kSlots), (v_idx / L::kSlots) & 1, wc);
+                v_ready = true;
+              }
+              if (!ok) continue;
+              tc_fence_after();
+              const uint64_t vd = v_desc(base + L::kKVOff + (v_idx % L::kSlots) * L::kTile, 0);
+#pragma unroll
+              for (int ks = 0; ks < kBlockN / 16; ++ks)
+                mma_ts(tmem + L::kColO0 + (uint32_t)D * t, tmem + L::kColP0 + 64u * t + 8u * ks,
+                       sdesc_advance(vd, (uint32_t)ks * 2048), idesc_pv, (j > 1 || ks > 0) ? 1u : 0u);
+              tc_commit(BAR(L::kPVDone + t));
+              if (j == nbt) tc_commit(BAR(L::kOFull + t));
+            }
+            if (!ok) break;
+            if (j == ui.K - 1) tc_commit(BAR(L::kQEmpty + qb));
+            if (j < ui.K) tc_commit(BAR(L::kKVEmpty + k_idx % L::kSlots));
+            if (j >= 1) tc_commit(BAR(L::kKVEmpty + v_idx % L::kSlots));
+          }
+          kv_iter = kv_base + 2 * ui.K;
+          o_uses0 += ui.nbk_0 > 0 ? 1u : 0u;
+          o_uses1 += ui.nbk_1 > 0 ? 1u : 0u;
+          continue;
+        }
         // Block-sparse: each query tile computes only the visited blocks it
         // attends (live); the other tile's blocks cost it no MMA and no
         // softmax.  Dense: tile t is live at visited block j iff j < nb_t.
@@ -457,8 +534,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + L::kColS0 + 128u * t;
     const uint32_t tO = tmem + lane_off + L::kColO0 + (uint32_t)D * t;
+    const uint32_t tP = kSepP ? tmem + lane_off + L::kColP0 + 64u * t : tS;   // where P goes
     const float sl2 = p.scale_log2;
     uint32_t s_cnt = 0, o_cnt = 0;
+    uint32_t p_stored = 0;   // P tiles written (separate-P pipeline: one P V product each)
     int unit_iter = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
@@ -487,6 +566,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < kBlockN / 32; ++c) tmem_ld32(tS + 32u * c, sr + 32 * c);
         tmem_wait_ld();
+        bool pv_seen = false;   // the previous P V product of this tile is known complete
+        if constexpr (kSepP) {
+          // S_t(j) is in registers: the MMA issuer may overwrite it with S_t(j+1)
+          tc_fence_before();
+          mbar_arrive(BAR(L::kSFree + t));
+        }
         float s[kBlockN];
 #pragma unroll
         for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(sr[c]);
@@ -523,6 +608,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           // instructions, so the whole warp takes the branch when any of its
           // rows needs it; rows that do not keep their max and use alpha = 1.
           if (__any_sync(0xffffffffu, need)) {
+            if constexpr (kSepP) {
+              // O must hold the previous P V product before it is rescaled
+              if (p_stored > 0) {
+                ok = warp_all(mbar_wait(BAR(L::kPVDone + t), (p_stored - 1) & 1, wc));
+                if (!ok) break;
+                tc_fence_after();
+              }
+              pv_seen = true;
+            }
             const float alpha = need ? ex2_approx(m_run - m_new) : 1.f;
             if (need) {
               l_run *= alpha;
@@ -543,6 +637,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;  // -inf row: every P is 0
         float ps[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pk_all[kSepP ? kBlockN / 2 : 1];   // separate P: stored after the wait below
 #pragma unroll
         for (int q = 0; q < kBlockN / 32; ++q) {
           uint32_t pk[16];
@@ -562,10 +657,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               pk[e] = pack2<BF16>(p0, p1);
             }
           }
-          if constexpr (FP8)
+          if constexpr (kSepP) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk_all[16 * q + e] = pk[e];
+          } else if constexpr (FP8) {
             tmem_st8(tS + 8u * q, pk);   // 32 keys = 8 columns of four e4m3
-          else
+          } else {
             tmem_st16(tS + 16u * q, pk);
+          }
+        }
+        if constexpr (kSepP) {
+          // the previous P of this tile must have been read by its P V product
+          if (p_stored > 0 && !pv_seen) {
+            ok = warp_all(mbar_wait(BAR(L::kPVDone + t), (p_stored - 1) & 1, wc));
+            if (!ok) break;
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int q = 0; q < kBlockN / 32; ++q) tmem_st16(tP + 16u * q, pk_all + 16 * q);
+          ++p_stored;
         }
         l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         tmem_wait_st();
@@ -642,10 +752,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 }
 
-template <int D, bool BF16, bool O32, bool CAUSAL, bool SPARSE>
+template <int D, bool BF16, bool O32, bool CAUSAL, bool SPARSE, bool SEPP = false>
 cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const FwdParams& p, int grid, cudaStream_t st) {
-  auto kern = fa_fwd_kernel<D, BF16, O32, CAUSAL, SPARSE>;
+  auto kern = fa_fwd_kernel<D, BF16, O32, CAUSAL, SPARSE, false, SEPP>;
   constexpr int smem = FwdLayout<D>::kAlloc;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -657,6 +767,13 @@ template <int D, bool BF16, bool O32>
 cudaError_t launch_fwd_c(bool causal, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const FwdParams& p, int grid, cudaStream_t st) {
   const bool sparse = p.bmask != nullptr;
+  // separate-P pipeline for short sequences at d = 64 (units of at most 16
+  // key blocks): measured faster at N = 1024, slower at N >= 4096
+  if constexpr (D == 64) {
+    if (!sparse && p.N <= 2048)
+      return causal ? launch_fwd_t<D, BF16, O32, true, false, true>(tq, tk, tv, p, grid, st)
+                    : launch_fwd_t<D, BF16, O32, false, false, true>(tq, tk, tv, p, grid, st);
+  }
   if (causal) return sparse ? launch_fwd_t<D, BF16, O32, true, true>(tq, tk, tv, p, grid, st)
                             : launch_fwd_t<D, BF16, O32, true, false>(tq, tk, tv, p, grid, st);
   return sparse ? launch_fwd_t<D, BF16, O32, false, true>(tq, tk, tv, p, grid, st)
