@@ -53,10 +53,15 @@ struct BwdLayout {
   static constexpr int kQT = BR * D * 2;           // Q or dO tile bytes
   static constexpr int kDS = kBlockN * BR * 2;     // dS^T tile bytes
   static constexpr int kStage = BR * D * 4;        // fp32 dQ staging bytes
-  static constexpr int kKOff = 0;
+  // K/V buffers: two at d = 64, so that the next unit's key/value tiles load
+  // while the current unit runs (units of short sequences are a few
+  // iterations long); the Q/dO ring is then 2 deep to stay within shared
+  // memory.  d = 128 (32 KB tiles): one K/V buffer, a 3-deep ring.
+  static constexpr int kKVBufs = (D == 64) ? 2 : 1;
+  static constexpr int kKOff = 0;                  // buffer b: K at b * 2 kKV, V after it
   static constexpr int kVOff = kKOff + kKV;
-  static constexpr int kStages = 3;               // Q / dO / LSE / D ring depth
-  static constexpr int kQOff = kVOff + kKV;        // [kStages]
+  static constexpr int kStages = (D == 64) ? 2 : 3;  // Q / dO / LSE / D ring depth
+  static constexpr int kQOff = kKVBufs * 2 * kKV;    // [kStages]
   static constexpr int kDOOff = kQOff + kStages * kQT;
   static constexpr int kDSOff = kDOOff + kStages * kQT;
   static constexpr int kStgOff = kDSOff + kDS;
@@ -64,8 +69,8 @@ struct BwdLayout {
   static constexpr int kVecStage = 2 * BR * 4;
   static constexpr int kBarOff = kVecOff + kStages * kVecStage;
   // barriers
-  static constexpr int kKVFull = 0, kKVEmpty = 1;
-  static constexpr int kQFull = 2;                 // [kStages]
+  static constexpr int kKVFull = 0, kKVEmpty = kKVBufs;   // [kKVBufs] each
+  static constexpr int kQFull = 2 * kKVBufs;             // [kStages]
   static constexpr int kQEmpty = kQFull + kStages;  // [kStages]
   static constexpr int kSFull = kQEmpty + kStages, kDPFull = kSFull + 1, kPFull = kSFull + 2;
   static constexpr int kDSFull = kSFull + 3, kDSEmpty = kSFull + 4, kDQFull = kSFull + 5;
@@ -209,8 +214,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::kMiscOff + 4);
 
   if (threadIdx.x == 0) {
-    mbar_init(BAR(L::kKVFull), 1);
-    mbar_init(BAR(L::kKVEmpty), 1);
+    for (int b = 0; b < L::kKVBufs; ++b) {
+      mbar_init(BAR(L::kKVFull + b), 1);
+      mbar_init(BAR(L::kKVEmpty + b), 1);
+    }
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(BAR(L::kQFull + s), 1);
       mbar_init(BAR(L::kQEmpty + s), 1);
@@ -251,17 +258,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_prefetch_desc(&tmDO);
       const uint64_t pol_kv = l2_policy_evict_first();
       const uint64_t pol_q = l2_policy_evict_last();
-      uint32_t unit_iter = 0, q_iter = 0;
+      uint32_t unit_iter = 0, q_iter = 0, kv_issued = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
         const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
-        if (unit_iter > 0 && !mbar_wait(BAR(L::kKVEmpty), (unit_iter - 1) & 1, wc)) { ok = false; break; }
-        mbar_arrive_expect_tx(BAR(L::kKVFull), 2 * L::kKV);
+        const uint32_t kb = unit_iter % L::kKVBufs, kuse = unit_iter / L::kKVBufs;
+        if (kuse > 0 && !mbar_wait(BAR(L::kKVEmpty + kb), (kuse - 1) & 1, wc)) { ok = false; break; }
+        mbar_arrive_expect_tx(BAR(L::kKVFull + kb), 2 * L::kKV);
+        const uint32_t kvb = base + kb * 2 * L::kKV;
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(base + L::kKOff + c * (kBlockN * 128), &tmK, BAR(L::kKVFull), c * 64, bu.jk * kBlockN, bu.kvbh, pol_kv);
-          tma_load_3d(base + L::kVOff + c * (kBlockN * 128), &tmV, BAR(L::kKVFull), c * 64, bu.jk * kBlockN, bu.kvbh, pol_kv);
+          tma_load_3d(kvb + L::kKOff + c * (kBlockN * 128), &tmK, BAR(L::kKVFull + kb), c * 64, bu.jk * kBlockN, bu.kvbh,
+                      pol_kv);
+          tma_load_3d(kvb + L::kVOff + c * (kBlockN * 128), &tmV, BAR(L::kKVFull + kb), c * 64, bu.jk * kBlockN, bu.kvbh,
+                      pol_kv);
         }
+        ++kv_issued;
         IterWin iw;
         for (int it = 0; it < bu.n_it; ++it) {
           if (!bactive<D, SPARSE>(iw, p, bu, it)) continue;
@@ -282,7 +294,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
       if (!ok) {
-        if (unit_iter > 0) mbar_wait_drain(BAR(L::kKVFull), (unit_iter - 1) & 1, p.wait_limit_ns);
+        // Let every copy already issued land before the CTA exits.
+        for (uint32_t b = 0; b < (uint32_t)L::kKVBufs; ++b) {
+          const uint32_t issued = kv_issued / L::kKVBufs + (b < kv_issued % L::kKVBufs ? 1u : 0u);
+          if (issued > 0) mbar_wait_drain(BAR(L::kKVFull + b), (issued - 1) & 1, p.wait_limit_ns);
+        }
         for (uint32_t s = 0; s < (uint32_t)L::kStages; ++s) {
           const uint32_t issued = q_iter / L::kStages + (s < q_iter % L::kStages ? 1u : 0u);
           if (issued > 0) mbar_wait_drain(BAR(L::kQFull + s), (issued - 1) & 1, p.wait_limit_ns);
@@ -300,8 +316,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
         const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
-        if (!mbar_wait(BAR(L::kKVFull), unit_iter & 1, wc)) { ok = false; break; }
-        const uint32_t sK = base + L::kKOff, sV = base + L::kVOff;
+        const uint32_t kb = unit_iter % L::kKVBufs;
+        if (!mbar_wait(BAR(L::kKVFull + kb), (unit_iter / L::kKVBufs) & 1, wc)) { ok = false; break; }
+        const uint32_t sK = base + kb * 2 * L::kKV + L::kKOff, sV = base + kb * 2 * L::kKV + L::kVOff;
         const uint64_t dK = kmaj<kBlockN>(sK, 0), dV = kmaj<kBlockN>(sV, 0), dKmn = mnmaj<kBlockN>(sK, 0);
         const uint64_t dDSmn = mnmaj<kBlockN>(base + L::kDSOff, 0);
         IterWin iw;  // walks forward only: the scan for the next iteration leads
@@ -380,7 +397,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         if (!ok) break;
         tc_commit(BAR(L::kAccFull));
-        tc_commit(BAR(L::kKVEmpty));
+        tc_commit(BAR(L::kKVEmpty + kb));
       }
       tc_commit(BAR(L::kDrain));
       mbar_wait_drain(BAR(L::kDrain), 0, p.wait_limit_ns);
