@@ -311,6 +311,7 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
   p.wait_limit_ns = wait_limit_ns();
+  p.debug_flags = g_debug_flags.load();
   p.bmask = bmask;
   p.bmask_stride = bmask_stride;
   if (!(p.status = status_ptr())) return FA_ERR_CUDA;

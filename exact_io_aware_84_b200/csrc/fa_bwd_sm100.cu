@@ -529,7 +529,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int c = 0; c < NC; ++c) tmem_st16(tS + HALF * w + 16u * c, pk + 16 * c);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(BAR(L::kPFull));
+        const bool withhold = (p.debug_flags & 2) && unit_iter == 0 && q_iter == 0 && tid256 == 0;
+        if (!withhold) mbar_arrive(BAR(L::kPFull));
         // dQ of the previous iteration (its MMA was issued after the previous
         // dS; its tensor-memory tile is reused by this iteration's dQ MMA)
         if (pend_qbh >= 0 && !(ok = stage_dq())) break;

@@ -69,6 +69,7 @@ struct BwdParams {
   float scale_log2;    // scale * log2(e)
   uint64_t wait_limit_ns;
   int* status;         // device status word
+  int debug_flags;     // bit 1: withhold one arrival (timeout test)
   const uint8_t* bmask;  // block sparsity as in FwdParams (nullptr = dense)
   long long bmask_stride;
 };

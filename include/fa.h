@@ -279,10 +279,10 @@ int fa_last_device_status(void* stream);
 /*
  * Diagnostics.  fa_debug_set_wait_limit_ms sets the per-wait limit used by
  * later launches (process-wide; ms >= 1).  fa_debug_set_flags sets
- * process-wide debug flags: bit 0 makes the forward kernel withhold one
- * pipeline arrival on its first tile, so that its bounded waits run out
- * and the launch ends with FA_ERR_TIMEOUT (used by the timeout test);
- * 0 restores normal operation.  Both return FA_OK or FA_ERR_INVALID_ARG.
+ * process-wide debug flags: bit 0 makes the forward kernel, bit 1 the
+ * backward's main kernel, withhold one pipeline arrival on its first tile,
+ * so that its bounded waits run out and the launch ends with FA_ERR_TIMEOUT
+ * (used by the timeout tests); 0 restores normal operation.  Both return FA_OK or FA_ERR_INVALID_ARG.
  */
 int fa_debug_set_wait_limit_ms(int ms);
 int fa_debug_set_flags(int flags);
