@@ -124,8 +124,27 @@ def load_library():
             fn = getattr(lib, name)
             fn.restype = res
             fn.argtypes = args
+        _apply_env(lib)
         _LIB = lib
     return _LIB
+
+
+def _apply_env(lib) -> None:
+    """Process-wide settings from the environment, applied once at load:
+    FA_WAIT_LIMIT (milliseconds, the bound on every pipeline wait inside a
+    kernel; default 1000) and FA_DEBUG (the debug flags of
+    fa_debug_set_flags; default 0)."""
+    for var, fn in (("FA_WAIT_LIMIT", lib.fa_debug_set_wait_limit_ms), ("FA_DEBUG", lib.fa_debug_set_flags)):
+        val = os.environ.get(var)
+        if val is None or val == "":
+            continue
+        try:
+            num = int(val, 0)
+        except ValueError as e:
+            raise ValueError(f"{var}={val!r} is not an integer") from e
+        st = fn(num)
+        if st != 0:
+            raise ValueError(f"{var}={val!r} rejected by the library (status {st})")
 
 
 def _status_name(status: int) -> str:

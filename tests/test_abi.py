@@ -170,3 +170,28 @@ def test_fp8_argument_errors():
     assert lib.fa_fwd_fp8(p, p, p, p, p, None, p, 16, 1, 1, 128, 128, 0.1, 0, 0, None) == fa.FA_ERR_WORKSPACE
     assert lib.fa_fwd_fp8(p, p, p, None, p, None, p, 1 << 30, 1, 1, 128, 128, 0.1, 0, 0, None) == fa.FA_ERR_INVALID_ARG
     assert lib.fa_fp8_quantize(None, p, p, None, p, 1 << 30, 1, 1, 128, 128, 0, None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_environment_settings_are_applied_and_checked(monkeypatch):
+    # FA_WAIT_LIMIT / FA_DEBUG are read when the library is loaded
+    monkeypatch.setenv("FA_WAIT_LIMIT", "250")
+    monkeypatch.setenv("FA_DEBUG", "0")
+    saved = fa._LIB
+    try:
+        fa._LIB = None
+        fa.load_library()
+        monkeypatch.setenv("FA_WAIT_LIMIT", "0")      # the library rejects ms < 1
+        fa._LIB = None
+        with pytest.raises(ValueError):
+            fa.load_library()
+        monkeypatch.setenv("FA_WAIT_LIMIT", "soon")
+        fa._LIB = None
+        with pytest.raises(ValueError):
+            fa.load_library()
+    finally:
+        monkeypatch.delenv("FA_WAIT_LIMIT")
+        monkeypatch.delenv("FA_DEBUG")
+        fa._LIB = None
+        fa.load_library()
+        fa.load_library().fa_debug_set_wait_limit_ms(1000)
+        fa._LIB = saved if saved is not None else fa._LIB
