@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t pol_q = l2_policy_evict_last();
       uint32_t unit_iter = 0, q_iter = 0, kv_issued = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
+      for (int k = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++k), ++unit_iter) {
         const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
         const uint32_t kb = unit_iter % L::kKVBufs, kuse = unit_iter / L::kKVBufs;
         if (kuse > 0 && !mbar_wait(BAR(L::kKVEmpty + kb), (kuse - 1) & 1, wc)) { ok = false; break; }
@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       constexpr uint32_t idesc_dq = make_idesc_f16(BF16, 128, 64, true, true);
       uint32_t unit_iter = 0, q_iter = 0, p_cnt = 0, ds_cnt = 0, dq_cnt = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
+      for (int k = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++k), ++unit_iter) {
         const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
         const uint32_t kb = unit_iter % L::kKVBufs;
         if (!mbar_wait(BAR(L::kKVFull + kb), (unit_iter / L::kKVBufs) & 1, wc)) { ok = false; break; }
@@ -487,7 +487,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       return warp_all(good);
     };
 
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
+    for (int k = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++k), ++unit_iter) {
       const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
       const int key = bu.jk * kBlockN + key_in;
       const bool key_ok = key < p.N;

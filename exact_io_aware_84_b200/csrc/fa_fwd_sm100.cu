@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const uint64_t pol_q = l2_policy_evict_first();
       uint32_t kv_iter = 0, unit_iter = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
+      for (int k = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++k), ++unit_iter) {
         const UnitInfo ui = decode_unit<CAUSAL, SPARSE>(u, p);
         const uint32_t qb = unit_iter % L::kQBufs, quse = unit_iter / L::kQBufs;
         if (quse > 0 && !mbar_wait(BAR(L::kQEmpty + qb), (quse - 1) & 1, wc)) { ok = false; break; }
@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       uint32_t p_cnt0 = 0, p_cnt1 = 0, o_uses0 = 0, o_uses1 = 0;
       uint32_t s_iss0 = 0, s_iss1 = 0;   // S MMAs issued per tile (separate-P pipeline)
       bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
+      for (int k = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++k), ++unit_iter) {
         const UnitInfo ui = decode_unit<CAUSAL, SPARSE>(u, p);
         const uint32_t qb = unit_iter % L::kQBufs;
         if (!mbar_wait(BAR(L::kQFull + qb), (unit_iter / L::kQBufs) & 1, wc)) { ok = false; break; }
@@ -540,7 +540,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint32_t p_stored = 0;   // P tiles written (separate-P pipeline: one P V product each)
     int unit_iter = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
+    for (int k = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++k), ++unit_iter) {
       const UnitInfo ui = decode_unit<CAUSAL, SPARSE>(u, p);
       if (ui.nb(t) == 0) continue;                 // query tile past the sequence end
       const int nb = ui.nbk(t);                    // key blocks this tile visits

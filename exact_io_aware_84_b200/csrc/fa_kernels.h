@@ -74,6 +74,16 @@ struct BwdParams {
   long long bmask_stride;
 };
 
+// The k-th work unit of this CTA in a persistent kernel: consecutive rounds
+// of gridDim.x units, taken in alternating directions (CTA c gets c, then
+// 2G-1-c, then 2G+c, ...).  Causal units are numbered longest first, so a CTA
+// that drew a long unit in one round draws a short one in the next; with a
+// plain round-robin the same CTAs would draw the longest unit of every round.
+__device__ __forceinline__ int unit_of(int k) {
+  const int g = (int)gridDim.x, c = (int)blockIdx.x;
+  return k * g + ((k & 1) ? g - 1 - c : c);
+}
+
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_fwd(int d, bool bf16, bool o32, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const FwdParams& p, int grid, cudaStream_t st);
