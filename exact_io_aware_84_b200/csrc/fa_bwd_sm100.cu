@@ -29,6 +29,8 @@
 //   warp  8     TMA producer      warp 9   MMA issuer      warps 10-11 idle
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "sm100_ptx.cuh"
 #include "fa_kernels.h"
 
@@ -506,23 +508,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ++s_cnt;
         tc_fence_after();
         const int q0 = i * BR + HALF * w;  // first query of this warpgroup's half
-        // P^T = exp2(S^T * scale*log2e - LSE*log2e), masked; kept packed
+        // P^T = exp2(S^T * scale*log2e - LSE*log2e), masked; kept packed.
+        // Only the key tile that holds the last keys (ragged) and, causal,
+        // tiles with a key after this half's first query need the mask: the
+        // test is uniform over the warpgroup, and the other tiles take the
+        // loop without the per-element compare and select.
+        const bool need_mask = (bu.jk + 1) * kBlockN > p.N || (CAUSAL && (bu.jk + 1) * kBlockN - 1 > q0);
         uint32_t pk[HALF / 2];
+        auto p_half = [&](auto masked) {
 #pragma unroll
-        for (int c = 0; c < NC; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tS + HALF * w + 32u * c, r);
-          tmem_wait_ld();
+          for (int c = 0; c < NC; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tS + HALF * w + 32u * c, r);
+            tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int qa = 32 * c + 2 * e;
-            float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * e]), sl2, -lse2[qa]));
-            float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * e + 1]), sl2, -lse2[qa + 1]));
-            if (!key_ok || (CAUSAL && key > q0 + qa)) p0 = 0.f;
-            if (!key_ok || (CAUSAL && key > q0 + qa + 1)) p1 = 0.f;
-            pk[16 * c + e] = pack2<BF16>(p0, p1);
+            for (int e = 0; e < 16; ++e) {
+              const int qa = 32 * c + 2 * e;
+              float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * e]), sl2, -lse2[qa]));
+              float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * e + 1]), sl2, -lse2[qa + 1]));
+              if constexpr (decltype(masked)::value) {
+                if (!key_ok || (CAUSAL && key > q0 + qa)) p0 = 0.f;
+                if (!key_ok || (CAUSAL && key > q0 + qa + 1)) p1 = 0.f;
+              }
+              pk[16 * c + e] = pack2<BF16>(p0, p1);
+            }
           }
-        }
+        };
+        if (need_mask)
+          p_half(std::true_type{});
+        else
+          p_half(std::false_type{});
         // packed P^T of this half -> columns [HALF*w, HALF*w + HALF/2) of the
         // S^T region, all of which this warpgroup has already read
 #pragma unroll
