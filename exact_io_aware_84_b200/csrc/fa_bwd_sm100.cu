@@ -10,7 +10,7 @@
 //                     loops over query tiles, keeps dK and dV in tensor memory,
 //                     adds each query tile's dQ into the fp32 accumulator with a
 //                     bulk shared->global reduce.
-//   3. fa_bwd_dq:     dQ = dtype(dQacc).
+//   3. fa_bwd_dq:     dQ = dtype(scale * dQacc).
 //
 // fa_bwd_main works transposed (keys on the 128 tensor-memory lanes):
 //   S^T = K_j Q_i^T, dP^T = V_j dO_i^T            (SS MMAs, M = 128 keys)
@@ -427,8 +427,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
 
     // Stage the pending dQ tile: read this warpgroup's 32 columns of it from
-    // tensor memory (scaled), write them into the fp32 staging tile, then one
-    // thread adds the whole tile into the global accumulator.
+    // tensor memory, write them into the fp32 staging tile, then one thread
+    // adds the whole tile into the global accumulator (the softmax scale is
+    // applied once, when the accumulator is converted).
     auto stage_dq = [&]() -> bool {
       // The two warpgroups meet on mbarriers with bounded waits, not on a
       // named barrier: if one of them has given up on a timeout, the other
@@ -465,15 +466,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int ch = 8 * w + ((e + key_in) & 7);
-          float4 f = make_float4(__uint_as_float(v[4 * e]) * p.scale, __uint_as_float(v[4 * e + 1]) * p.scale,
-                                 __uint_as_float(v[4 * e + 2]) * p.scale, __uint_as_float(v[4 * e + 3]) * p.scale);
+          float4 f = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                 __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
           *reinterpret_cast<float4*>(stage + key_in * 64 + 4 * ch) = f;
         }
       } else {
         // lane = dim key_in, columns = queries 32w..32w+31: column key_in of
         // the [64 queries][128 dims] tile
 #pragma unroll
-        for (int q = 0; q < 32; ++q) stage[(32 * w + q) * 128 + key_in] = __uint_as_float(v[q]) * p.scale;
+        for (int q = 0; q < 32; ++q) stage[(32 * w + q) * 128 + key_in] = __uint_as_float(v[q]);
       }
       fence_async_smem();
       mbar_arrive(BAR(L::kStgDone));
@@ -501,8 +502,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t st = q_iter % L::kStages;
         ok = warp_all(mbar_wait(BAR(L::kQFull + st), (q_iter / L::kStages) & 1, wc));
         if (!ok) break;
-        const float* lse2 = reinterpret_cast<const float*>(gbase + L::kVecOff + st * L::kVecStage) + HALF * w;
-        const float* dvec = lse2 + BR;
+        // this half's LSE*log2e and D, read four at a time (16-byte aligned)
+        const float4* lse2 = reinterpret_cast<const float4*>(gbase + L::kVecOff + st * L::kVecStage) + HALF * w / 4;
+        const float4* dvec = lse2 + BR / 4;
         ok = warp_all(mbar_wait(BAR(L::kSFull), s_cnt & 1, wc));
         if (!ok) break;
         ++s_cnt;
@@ -521,11 +523,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             uint32_t r[32];
             tmem_ld32(tS + HALF * w + 32u * c, r);
             tmem_wait_ld();
+            float4 lq;
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int qa = 32 * c + 2 * e;
-              float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * e]), sl2, -lse2[qa]));
-              float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * e + 1]), sl2, -lse2[qa + 1]));
+              if ((e & 1) == 0) lq = lse2[qa >> 2];
+              float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * e]), sl2, -((e & 1) ? lq.z : lq.x)));
+              float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * e + 1]), sl2, -((e & 1) ? lq.w : lq.y)));
               if constexpr (decltype(masked)::value) {
                 if (!key_ok || (CAUSAL && key > q0 + qa)) p0 = 0.f;
                 if (!key_ok || (CAUSAL && key > q0 + qa + 1)) p1 = 0.f;
@@ -569,9 +573,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_ld32(tDP + HALF * w + 32u * c, r);
           tmem_wait_ld();
           uint32_t dsk[16];
+          float4 dq4;
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int qa = 32 * c + 2 * e;
+            if ((e & 1) == 0) dq4 = dvec[qa >> 2];
             const uint32_t pp = pk[16 * c + e];
             float p0, p1;
             if constexpr (BF16) {
@@ -582,8 +588,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               p0 = __low2float(h);
               p1 = __high2float(h);
             }
-            const float ds0 = p0 * (__uint_as_float(r[2 * e]) - dvec[qa]);
-            const float ds1 = p1 * (__uint_as_float(r[2 * e + 1]) - dvec[qa + 1]);
+            const float ds0 = p0 * (__uint_as_float(r[2 * e]) - ((e & 1) ? dq4.z : dq4.x));
+            const float ds1 = p1 * (__uint_as_float(r[2 * e + 1]) - ((e & 1) ? dq4.w : dq4.y));
             dsk[e] = pack2<BF16>(ds0, ds1);
           }
           tmem_st16(tDP + HALF * w + 16u * c, dsk);
@@ -738,7 +744,9 @@ __global__ void __launch_bounds__(256) fa_bwd_dq(const BwdParams p) {
   const size_t bh = row / p.N, n = row % p.N;
   const float4* src = reinterpret_cast<const float4*>(p.dq_acc + (bh * p.n_pad + n) * D + g * 8);
   const float4 a = src[0], b = src[1];
-  uint4 w = make_uint4(pack2<BF16>(a.x, a.y), pack2<BF16>(a.z, a.w), pack2<BF16>(b.x, b.y), pack2<BF16>(b.z, b.w));
+  const float c = p.scale;  // the accumulator holds dS K without the softmax scale
+  uint4 w = make_uint4(pack2<BF16>(a.x * c, a.y * c), pack2<BF16>(a.z * c, a.w * c), pack2<BF16>(b.x * c, b.y * c),
+                       pack2<BF16>(b.z * c, b.w * c));
   reinterpret_cast<uint4*>(p.dq)[idx] = w;
 }
 
