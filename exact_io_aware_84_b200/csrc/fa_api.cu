@@ -319,7 +319,7 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   const size_t vec_bytes = ((size_t)bh * p.n_pad * sizeof(float) + 255) / 256 * 256;
   p.dq_acc = static_cast<float*>(workspace);
   p.dvec = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + acc_bytes);
-  p.lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + acc_bytes + vec_bytes);
+  p.nlse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + acc_bytes + vec_bytes);
   CUtensorMap tq, tk, tv, tdo;
   const int q_rows = (d == 64) ? 128 : 64;  // backward query tile (see fa_bwd_sm100.cu)
   if (encode_tile_map(&tq, q, bh, N, d, bf16, q_rows) != FA_OK ||

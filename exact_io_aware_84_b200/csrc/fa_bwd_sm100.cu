@@ -5,7 +5,7 @@
 // With dP = dO V^T, D_i = sum_c dO_ic O_ic and dS = P o (dP - D):
 //   dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
 // Three launches:
-//   1. fa_bwd_prep:   D_i, LSE_i * log2(e) (+inf on padding rows), zero dQacc.
+//   1. fa_bwd_prep:   D_i, -LSE_i * log2(e) (-inf on padding rows), zero dQacc.
 //   2. fa_bwd_main:   one CTA per (batch*head, 128-key tile) unit, persistent;
 //                     loops over query tiles, keeps dK and dV in tensor memory,
 //                     adds each query tile's dQ into the fp32 accumulator with a
@@ -67,7 +67,7 @@ struct BwdLayout {
   static constexpr int kDOOff = kQOff + kStages * kQT;
   static constexpr int kDSOff = kDOOff + kStages * kQT;
   static constexpr int kStgOff = kDSOff + kDS;
-  static constexpr int kVecOff = kStgOff + kStage;  // [kStages] x (lse2[BR], dvec[BR])
+  static constexpr int kVecOff = kStgOff + kStage;  // [kStages] x (nlse2[BR], dvec[BR])
   static constexpr int kVecStage = 2 * BR * 4;
   static constexpr int kBarOff = kVecOff + kStages * kVecStage;
   // barriers
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tma_load_3d(base + L::kDOOff + st * L::kQT + c * (BR * 128), &tmDO, fb, c * 64, i * BR, qbh, pol_q);
           }
           const size_t row0 = (size_t)qbh * p.n_pad + (size_t)i * BR;
-          bulk_load(base + L::kVecOff + st * L::kVecStage, p.lse2 + row0, BR * 4, fb);
+          bulk_load(base + L::kVecOff + st * L::kVecStage, p.nlse2 + row0, BR * 4, fb);
           bulk_load(base + L::kVecOff + st * L::kVecStage + BR * 4, p.dvec + row0, BR * 4, fb);
           ++q_iter;
         }
@@ -502,9 +502,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t st = q_iter % L::kStages;
         ok = warp_all(mbar_wait(BAR(L::kQFull + st), (q_iter / L::kStages) & 1, wc));
         if (!ok) break;
-        // this half's LSE*log2e and D, read four at a time (16-byte aligned)
-        const float4* lse2 = reinterpret_cast<const float4*>(gbase + L::kVecOff + st * L::kVecStage) + HALF * w / 4;
-        const float4* dvec = lse2 + BR / 4;
+        // this half's -LSE*log2e and D, read four at a time (16-byte aligned)
+        const float4* nlse2 = reinterpret_cast<const float4*>(gbase + L::kVecOff + st * L::kVecStage) + HALF * w / 4;
+        const float4* dvec = nlse2 + BR / 4;
+        const uint64_t sl2x2 = f2_pack(sl2, sl2);
         ok = warp_all(mbar_wait(BAR(L::kSFull), s_cnt & 1, wc));
         if (!ok) break;
         ++s_cnt;
@@ -527,9 +528,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int qa = 32 * c + 2 * e;
-              if ((e & 1) == 0) lq = lse2[qa >> 2];
-              float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * e]), sl2, -((e & 1) ? lq.z : lq.x)));
-              float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * e + 1]), sl2, -((e & 1) ? lq.w : lq.y)));
+              if ((e & 1) == 0) lq = nlse2[qa >> 2];
+              // both exponents of the pair in one two-wide fma
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), sl2x2,
+                               (e & 1) ? f2_pack(lq.z, lq.w) : f2_pack(lq.x, lq.y)),
+                        x0, x1);
+              float p0 = ex2_approx(x0);
+              float p1 = ex2_approx(x1);
               if constexpr (decltype(masked)::value) {
                 if (!key_ok || (CAUSAL && key > q0 + qa)) p0 = 0.f;
                 if (!key_ok || (CAUSAL && key > q0 + qa + 1)) p1 = 0.f;
@@ -588,8 +594,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               p0 = __low2float(h);
               p1 = __high2float(h);
             }
-            const float ds0 = p0 * (__uint_as_float(r[2 * e]) - ((e & 1) ? dq4.z : dq4.x));
-            const float ds1 = p1 * (__uint_as_float(r[2 * e + 1]) - ((e & 1) ? dq4.w : dq4.y));
+            // dS = P (dP - D) for the pair in two two-wide instructions
+            float ds0, ds1;
+            f2_unpack(f2_mul(f2_pack(p0, p1),
+                             f2_sub(f2_pack(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])),
+                                    (e & 1) ? f2_pack(dq4.z, dq4.w) : f2_pack(dq4.x, dq4.y))),
+                      ds0, ds1);
             dsk[e] = pack2<BF16>(ds0, ds1);
           }
           tmem_st16(tDP + HALF * w + 16u * c, dsk);
@@ -722,9 +732,9 @@ __global__ void __launch_bounds__(256) fa_bwd_prep(const BwdParams p) {
       if (sub == 0) {
         p.dvec[prow] = acc;
         // padding rows and rows with no kept key (LSE = -inf, block-sparse)
-        // get +inf, so that any P recomputed for them is 0
+        // get -inf, so that any P recomputed for them is 0
         const float l = row < p.N ? p.lse[(size_t)bh * p.N + row] : -INFINITY;
-        p.lse2[prow] = l > -INFINITY ? l * 1.4426950408889634f : INFINITY;
+        p.nlse2[prow] = l > -INFINITY ? -(l * 1.4426950408889634f) : -INFINITY;
       }
       float4* acc_row = reinterpret_cast<float4*>(p.dq_acc + prow * D) + 2 * sub;
       acc_row[0] = make_float4(0.f, 0.f, 0.f, 0.f);

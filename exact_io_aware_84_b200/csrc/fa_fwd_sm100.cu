@@ -629,26 +629,35 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               uint32_t o[32];
               tmem_ld32(tO + 32u * c, o);
               tmem_wait_ld();
+              const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              for (int e = 0; e < 16; ++e) {
+                float lo, hi;
+                f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), a2), lo, hi);
+                o[2 * e] = __float_as_uint(lo);
+                o[2 * e + 1] = __float_as_uint(hi);
+              }
               tmem_st32(tO + 32u * c, o);
             }
           }
         }
         const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;  // -inf row: every P is 0
-        float ps[4] = {0.f, 0.f, 0.f, 0.f};
+        // exponents and row sums of key pairs with the two-wide fp32
+        // instructions: four pair accumulators (eight partial sums)
+        const uint64_t cl2x2 = f2_pack(c_l2, c_l2), nm2 = f2_pack(neg_m, neg_m);
+        uint64_t ps2[4] = {0ull, 0ull, 0ull, 0ull};
         uint32_t pk_all[kSepP ? kBlockN / 2 : 1];   // separate P: stored after the wait below
 #pragma unroll
         for (int q = 0; q < kBlockN / 32; ++q) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float x0 = fmaf(s[32 * q + 2 * e], c_l2, neg_m);
-            const float x1 = fmaf(s[32 * q + 2 * e + 1], c_l2, neg_m);
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(s[32 * q + 2 * e], s[32 * q + 2 * e + 1]), cl2x2, nm2), x0, x1);
             const bool poly = (poly_pair_mask<D, FP8>() >> (e & 7)) & 1u;
             const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
             const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
-            ps[e & 3] += p0 + p1;
+            ps2[e & 3] = f2_add(ps2[e & 3], f2_pack(p0, p1));
             if constexpr (FP8) {
               // two e4m3 per 16 bits; element pairs (2e, 2e + 1) of 32 keys
               const uint32_t h = pack_e4m3x2(p0, p1);
@@ -677,7 +686,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int q = 0; q < kBlockN / 32; ++q) tmem_st16(tP + 16u * q, pk_all + 16 * q);
           ++p_stored;
         }
-        l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+        {
+          float a0, a1, b0, b1;
+          f2_unpack(f2_add(ps2[0], ps2[1]), a0, a1);
+          f2_unpack(f2_add(ps2[2], ps2[3]), b0, b1);
+          l_run += (a0 + b0) + (a1 + b1);
+        }
         tmem_wait_st();
         tc_fence_before();
         const bool withhold = (p.debug_flags & 1) && unit_iter == 0 && j == 0 && t == 0;

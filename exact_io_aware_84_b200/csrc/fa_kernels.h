@@ -58,7 +58,7 @@ struct BwdParams {
   void* dv;            // [B*H, N, D]
   float* dq_acc;       // [B*H, n_pad, D] fp32 workspace
   float* dvec;         // [B*H, n_pad] fp32 workspace (D_i)
-  float* lse2;         // [B*H, n_pad] fp32 workspace (LSE_i * log2 e; +inf on padding)
+  float* nlse2;        // [B*H, n_pad] fp32 workspace (-LSE_i * log2 e; -inf on padding)
   int N;
   int n_pad;           // ceil(N / 128) * 128
   int bh;              // B*H (query heads)

@@ -92,7 +92,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
  * Bytes of device workspace fa_bwd needs for these sizes: a float32 dQ
  * accumulator of B*H*ceil(N/128)*128*d elements, then two float32 row
  * vectors of B*H*ceil(N/128)*128 elements (D_i = sum_c dO_ic O_ic, and
- * LSE_i * log2(e)), each section rounded up to 256 bytes.  Returns 0 for
+ * -LSE_i * log2(e)), each section rounded up to 256 bytes.  Returns 0 for
  * invalid sizes.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
