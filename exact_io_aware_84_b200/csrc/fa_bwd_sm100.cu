@@ -248,6 +248,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{p.wait_limit_ns, abort_flag, p.status};
+  // nothing above touched global memory; D, -LSE*log2e and the zeroed dQ
+  // accumulator come from the preparation kernel
+  grid_dependency_wait();
+  grid_dependents_launch();
   if (warp >= 8) regs_dec<kBRegsNarrow>();
   else regs_inc<kBRegsWide>();
 
@@ -677,6 +681,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // over the row groups.  O is read as 16-bit, or as fp32 for the O32 codes.
 template <int D, bool BF16, bool O32>
 __global__ void __launch_bounds__(256) fa_bwd_prep(const BwdParams p) {
+  grid_dependency_wait();  // O, dO and LSE from the kernels before; the workspace free again
+  grid_dependents_launch();
   constexpr int L = D / 8;            // lanes per row
   constexpr int RPW = 32 / L;         // rows per warp pass
   const int lane = threadIdx.x & 31;
@@ -746,6 +752,8 @@ __global__ void __launch_bounds__(256) fa_bwd_prep(const BwdParams p) {
 // dQ = dtype(dQacc) for the real rows.  One thread per 8 elements.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256) fa_bwd_dq(const BwdParams p) {
+  grid_dependency_wait();  // every reduce into the accumulator has landed
+  grid_dependents_launch();
   const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;  // 8-element group
   const size_t groups = (size_t)p.bh * p.N * (D / 8);
   if (idx >= groups) return;
@@ -769,11 +777,9 @@ cudaError_t launch_bwd_t(bool o32, const CUtensorMap& tq, const CUtensorMap& tk,
     const long long groups = ((long long)p.bh * p.n_pad + 32 / (D / 8) - 1) / (32 / (D / 8));
     const long long want = (groups + 7) / 8;
     const int blocks = (int)(want < 148LL * 16 ? want : 148LL * 16);
-    if (o32)
-      fa_bwd_prep<D, BF16, true><<<blocks, 256, 0, st>>>(p);
-    else
-      fa_bwd_prep<D, BF16, false><<<blocks, 256, 0, st>>>(p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = o32 ? launch_chained(fa_bwd_prep<D, BF16, true>, dim3(blocks), dim3(256), 0, st, p)
+                        : launch_chained(fa_bwd_prep<D, BF16, false>, dim3(blocks), dim3(256), 0, st, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   {
@@ -781,15 +787,15 @@ cudaError_t launch_bwd_t(bool o32, const CUtensorMap& tq, const CUtensorMap& tk,
     constexpr int smem = BwdLayout<D>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kBwdThreads, smem, st>>>(tq, tk, tv, tdo, p);
-    e = cudaGetLastError();
+    e = launch_chained(kern, dim3(grid), dim3(kBwdThreads), smem, st, tq, tk, tv, tdo, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   {
     const long long groups = (long long)p.bh * p.N * (D / 8);
     const int blocks = (int)((groups + 255) / 256);
-    fa_bwd_dq<D, BF16><<<blocks, 256, 0, st>>>(p);
-    return cudaGetLastError();
+    cudaError_t e = launch_chained(fa_bwd_dq<D, BF16>, dim3(blocks), dim3(256), 0, st, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
   }
 }
 

@@ -272,6 +272,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{p.wait_limit_ns, abort_flag, p.status};
+  // nothing above touched global memory: from here on the previous kernel's
+  // results are needed (and its reads of O and LSE must be over)
+  grid_dependency_wait();
+  grid_dependents_launch();
 
   if (warp >= 8) regs_dec<kRegsOther>();
   if (warp == kProducerWarp) {
@@ -773,8 +777,8 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   constexpr int smem = FwdLayout<D>::kAlloc;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kFwdThreads, smem, st>>>(tq, tk, tv, p);
-  return cudaGetLastError();
+  e = launch_chained(kern, dim3(grid), dim3(kFwdThreads), smem, st, tq, tk, tv, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int D, bool BF16, bool O32>

@@ -6,7 +6,31 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <utility>
+
 namespace fa {
+
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel in the stream is finishing, so that its launch
+// and prologue (barrier setup, tensor-memory allocation) overlap that tail.
+// Every kernel launched this way executes griddepcontrol.wait before its
+// first access to global memory, which returns once the previous grid has
+// completed and its writes are visible.
+template <typename... Params, typename... Args>
+inline cudaError_t launch_chained(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                  Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 constexpr int kBlockM = 128;  // query rows per Q tile (tcgen05 M)
 constexpr int kBlockN = 128;  // keys per K/V tile

@@ -345,6 +345,16 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   return r;
 }
 
+// Programmatic dependent launch.  grid_dependency_wait returns once the grid
+// this one was chained to (the previous kernel in the stream) has completed
+// and its memory operations are visible; a kernel launched without the
+// chaining attribute returns at once.  grid_dependents_launch lets the next
+// chained kernel in the stream be scheduled.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Two-wide fp32 arithmetic of sm_100 (one instruction for a pair of floats,
 // each lane rounded to nearest as by the scalar instruction).  A pair lives
 // in a 64-bit register: lo in bits 0-31.
