@@ -539,7 +539,7 @@ def _target_fwd(fa, torch, dev, stream, flush, peaks, args):
             "target_frac": 0.60}
 
 
-def _e2e(fa, torch, w, x, dev, stream, flops, world, args):
+def _e2e(fa, torch, w, x, dev, stream, flops, world, args, outputs=None):
     """The metric end to end through the public calls: every step copies its
     inputs from pinned host memory to the device, runs fa_fwd (and fa_bwd)
     and copies all of its outputs (O, LSE, and dQ, dK, dV) back to pinned host
@@ -548,7 +548,8 @@ def _e2e(fa, torch, w, x, dev, stream, flops, world, args):
     link carries both directions at once).  Device buffers alternate between
     two slots, ordered by events, so no copy touches a buffer a kernel still
     uses.  The timed region runs from before the first upload to after the
-    last download."""
+    last download.  ``outputs``, when a dict, receives the host copies of the
+    last step's results."""
     pin = {k: v.pin_memory() for k, v in x.items()}
     B, H, N, d = w.B, w.H, w.N, w.d
     out_names = ["o", "lse"] + (["dq", "dk", "dv"] if w.backward else [])
@@ -612,6 +613,8 @@ def _e2e(fa, torch, w, x, dev, stream, flops, world, args):
     e.record(cout)   # after the last download, which waited for all the rest
     torch.cuda.synchronize()
     ms = _max_over_ranks(s.elapsed_time(e), world) / args.steps
+    if outputs is not None:
+        outputs.update(host_out[(k - 1) % 2])
     return {"value": flops * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "pipeline": "copy-in / compute / copy-out streams"}
 
