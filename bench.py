@@ -486,10 +486,10 @@ def _attended_pairs(mask, N, causal):
 
 def _memory_vs_n(fa, torch, dev, stream):
     """Peak device memory of one forward + backward at d=128, B=2, H=16 for
-    N in {2048, 8192, 16384} (every buffer the call needs: inputs, outputs,
-    workspace), next to the score matrix standard attention would hold
-    (B H N^2 x 2 bytes).  Linear in N: the kernels never store an N x N
-    matrix."""
+    N in {2048, 8192, 16384}, and at the trading-day shape (every buffer the
+    call needs: inputs, outputs, workspace), next to the score matrix
+    standard attention would hold (B H N^2 x 2 bytes).  Linear in N: the
+    kernels never store an N x N matrix."""
     from exact_io_aware_84_b200.metrics import score_matrix_bytes
     out = {"B": 2, "H": 16, "d": 128, "N": [], "peak_bytes": [], "score_matrix_bytes_bf16": []}
     for n in (2048, 8192, 16384):
@@ -509,6 +509,20 @@ def _memory_vs_n(fa, torch, dev, stream):
     per_n = [b / n for b, n in zip(out["peak_bytes"], out["N"])]
     out["bytes_per_token"] = per_n
     out["linear_in_n"] = max(per_n) / min(per_n) < 1.05
+    # the one-trading-day shape (B=1, H=12, N=23400, d=64, causal), one point
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    torch.cuda.reset_peak_memory_stats(dev)
+    base = torch.cuda.memory_allocated(dev)
+    B, H, n, d = 1, 12, 23400, 64
+    q, k, v, do = (torch.randn((B, H, n, d), device=dev, dtype=torch.bfloat16) for _ in range(4))
+    o, lse = fa.fa_fwd(q, k, v, causal=True, stream=stream)
+    fa.fa_bwd(q, k, v, o, do, lse, causal=True, stream=stream)
+    torch.cuda.synchronize()
+    peak = int(torch.cuda.max_memory_allocated(dev) - base)
+    out["trading_day"] = {"B": B, "H": H, "N": n, "d": d, "causal": True, "peak_bytes": peak,
+                          "bytes_per_token": peak / n, "score_matrix_bytes_bf16": score_matrix_bytes(B, H, n, 2)}
+    del q, k, v, do, o, lse
     return out
 
 
