@@ -17,6 +17,7 @@ from .attention import (  # noqa: F401
     blocksparse_bwd_ref,
     merge_partials_ref,
     attn_bwd_partial_ref,
+    attn_dq_rows_ref,
     ring_fwd_ref,
     ring_bwd_ref,
 )

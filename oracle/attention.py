@@ -27,8 +27,9 @@ What it computes (all in float64, on whatever arrays it is handed):
 * ``online_fwd_ref`` -- the online-softmax re-association, one key/value block
   at a time: running row max m, running sum l, unnormalised accumulator O~;
   when the max grows, O~ and l are rescaled by exp(m_old - m_new); O = O~ / l
-  at the end.  Source: ultralytics.com glossary "Flash Attention", the
-  streaming loop of its code listing, and marketmaker.cc section "Online
+  at the end.  Source: ultralytics.com glossary "Flash Attention", section
+  "How Flash Attention works" (streaming blocks with a running max and
+  sum), and marketmaker.cc section "Online
   softmax recurrence" (whose displayed equations were lost in extraction; they
   are reconstructed from its prose, which says that whenever a block raises
   the running maximum the output accumulated so far is multiplied by
@@ -63,6 +64,10 @@ What it computes (all in float64, on whatever arrays it is handed):
   The gradient of a chunk pair uses the full row statistics (the merged LSE
   and O): P = exp(S - LSE), D = rowsum(dO o O), and the per-pair dQ, dK, dV
   sum to the full gradient.
+* ``attn_dq_rows_ref`` -- dQ of selected query rows only (each row's dQ
+  needs only that row's P, dP and D), with an optional stored O standing in
+  for the exact O inside D = rowsum(dO o O): the tool that measures how much
+  of the gradient error comes from the storage precision of O alone.
 * ``fa1_fwd_ref`` -- the per-step-normalised loop of the marketmaker.cc
   section "The Flash Attention algorithm" (query blocks outer, key/value blocks
   inner, O normalised by the running sum after every block).
@@ -95,6 +100,7 @@ __all__ = [
     "blocksparse_fwd_ref",
     "merge_partials_ref",
     "attn_bwd_partial_ref",
+    "attn_dq_rows_ref",
     "ring_fwd_ref",
     "ring_bwd_ref",
     "blocksparse_bwd_ref",
@@ -227,41 +233,47 @@ def attn_bwd_ref(q, k, v, do, scale, causal=False, row_chunk=1024):
 
 
 def online_fwd_ref(q, k, v, scale, causal=False, block=128, dtype=np.float64):
-    """Online-softmax forward for one head, streaming key/value blocks.
+    """Online-softmax forward for one head: the key/value sequence is consumed
+    one block at a time and never seen again.
 
-    All query rows are processed against one key/value block at a time.  After
-    block j:  m_j = max(m_{j-1}, rowmax S_j);  l_j = e^{m_{j-1}-m_j} l_{j-1} +
-    rowsum e^{S_j - m_j};  O~_j = e^{m_{j-1}-m_j} O~_{j-1} + e^{S_j - m_j} V_j.
-    Finally O = O~ / l and LSE = m + ln l.  ``dtype`` lets the same steps run
-    in float32 (the glossary's own precision) for its worked error figure.
+    State per query row i, after the first j key blocks: the largest scaled
+    score seen so far (mu), the sum of exp(score - mu) over those keys (ell),
+    and the matching unnormalised output, sum of exp(score - mu) v_key (acc).
+    Block j+1 moves the reference point to mu' = max(mu, its own row max);
+    the old state is carried over by the factor exp(mu - mu') (zero while mu
+    is still -inf), and the block adds its own exp(score - mu') terms.  At the
+    end O = acc / ell and LSE = mu + ln ell.  ``dtype`` selects the working
+    precision (float32 reproduces the glossary's worked error figure).
     """
-    q = np.asarray(q, dtype=dtype)
-    k = np.asarray(k, dtype=dtype)
-    v = np.asarray(v, dtype=dtype)
-    n, nk = q.shape[0], k.shape[0]
-    sc = dtype(scale)
-    row_max = np.full((n, 1), -np.inf, dtype=dtype)
-    row_sum = np.zeros((n, 1), dtype=dtype)
-    out = np.zeros((n, v.shape[1]), dtype=dtype)
-    rows = np.arange(n)
-    for start in range(0, nk, block):
-        stop = min(nk, start + block)
-        scores = (q @ k[start:stop].T) * sc
+    dt = np.dtype(dtype).type
+    Q = np.asarray(q, dtype=dt)
+    K = np.asarray(k, dtype=dt)
+    V = np.asarray(v, dtype=dt)
+    n_q, n_k = Q.shape[0], K.shape[0]
+    query_pos = np.arange(n_q)[:, None]
+    mu = np.full((n_q, 1), -np.inf, dtype=dt)
+    ell = np.zeros((n_q, 1), dtype=dt)
+    acc = np.zeros((n_q, V.shape[1]), dtype=dt)
+    for j0 in range(0, n_k, block):
+        j1 = min(n_k, j0 + block)
+        sc = (Q @ K[j0:j1].T) * dt(scale)
         if causal:
-            cols = np.arange(start, stop)
-            scores = np.where(cols[None, :] > rows[:, None], -np.inf, scores)
-        new_max = np.maximum(row_max, scores.max(axis=-1, keepdims=True))
-        safe = np.where(np.isfinite(new_max), new_max, 0.0).astype(dtype)
+            sc = np.where(np.arange(j0, j1)[None, :] > query_pos, -np.inf, sc)
+        mu_new = np.maximum(mu, sc.max(axis=1, keepdims=True))
+        seen = np.isfinite(mu_new)                # at least one unmasked key so far
+        ref = np.where(seen, mu_new, 0.0).astype(dt)
         with np.errstate(invalid="ignore"):
-            rescale = np.where(np.isfinite(new_max), np.exp(row_max - safe), 0.0).astype(dtype)
-        probs = np.exp(scores - safe)
-        row_sum = row_sum * rescale + probs.sum(axis=-1, keepdims=True)
-        out = out * rescale + probs @ v[start:stop]
-        row_max = new_max
-    with np.errstate(divide="ignore", invalid="ignore"):
-        o = np.where(row_sum > 0, out / np.where(row_sum > 0, row_sum, 1), 0.0)
-        lse = np.where(row_sum > 0, row_max + np.log(np.where(row_sum > 0, row_sum, 1)), -np.inf)
-    return o.astype(dtype), lse[:, 0].astype(dtype)
+            carry = np.where(seen, np.exp(mu - ref), 0.0).astype(dt)
+        w = np.exp(sc - ref)                      # masked entries give exp(-inf) = 0
+        ell = carry * ell + w.sum(axis=1, keepdims=True)
+        acc = carry * acc + w @ V[j0:j1]
+        mu = mu_new
+    live = ell > 0
+    ell_safe = np.where(live, ell, 1)
+    o = np.where(live, acc / ell_safe, 0.0)
+    with np.errstate(divide="ignore"):
+        lse = np.where(live, mu + np.log(ell_safe), -np.inf)
+    return o.astype(dt), lse[:, 0].astype(dt)
 
 
 def fa1_fwd_ref(q, k, v, scale, causal=False, block_r=128, block_c=128):
@@ -393,6 +405,35 @@ def blocksparse_bwd_ref(q, k, v, do, scale, causal, block_mask, block=128):
         dk[h] = float(scale) * (ds.T @ qf[h])
     shp = lambda x, ref: x.reshape(lead + ref.shape[-2:])
     return shp(dq, q), shp(dk, k), shp(dv, v)
+
+
+def attn_dq_rows_ref(q, k, v, do, scale, causal=False, rows=None, o_for_d=None):
+    """dQ of the selected query rows of one head (q, k, v, do: [N, d]).
+
+    dQ_i depends on row i alone: P_i = softmax(S_i) (two-pass), O_i = P_i V,
+    dP_i = dO_i V^T, D_i = sum_c dO_ic O_ic, dS_i = P_i o (dP_i - D_i),
+    dQ_i = scale dS_i K.  ``o_for_d``, when given, replaces the exact O_i in
+    D_i only -- the O a backward reads back from storage -- so that the effect
+    of storing O at a lower precision can be isolated with every other step
+    exact.  It is a function applied to the exact fp64 O of the rows (the
+    storage rounding), or a list of such functions and None (one dQ per
+    entry, all from the same scores).  Returns [len(rows), d] float64, or a
+    list of them.
+    """
+    k, v = _f64(k), _f64(v)
+    do = _f64(do)
+    s, rows = attn_scores_ref(q, k, scale, causal, rows=rows)
+    _, p = _two_pass(s)
+    o = p @ v
+    d_o = do[rows]
+    dp = d_o @ v.T
+    many = isinstance(o_for_d, (list, tuple))
+    outs = []
+    for store in (o_for_d if many else [o_for_d]):
+        o_d = o if store is None else _f64(store(o))
+        D = np.sum(d_o * o_d, axis=-1, keepdims=True)
+        outs.append(float(scale) * ((p * (dp - D)) @ k))
+    return outs if many else outs[0]
 
 
 def merge_partials_ref(o_a, lse_a, o_b, lse_b):

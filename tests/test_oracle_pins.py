@@ -25,8 +25,8 @@ from oracle import (attn_bwd_ref, attn_fwd_ref, attn_fwd_rows_ref,
                     attn_probs_ref, attn_scores_ref, fa1_fwd_ref,
                     blocksparse_bwd_ref, blocksparse_fwd_ref,
                     gqa_bwd_ref, gqa_fwd_ref, online_fwd_ref,
-                    attn_bwd_partial_ref, merge_partials_ref, ring_bwd_ref,
-                    ring_fwd_ref)
+                    attn_bwd_partial_ref, attn_dq_rows_ref, merge_partials_ref,
+                    ring_bwd_ref, ring_fwd_ref)
 from exact_io_aware_84_b200.metrics import score_matrix_bytes
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -295,6 +295,34 @@ def test_gradient_matches_finite_differences(n, d, causal):
         rel = np.linalg.norm(ana - num) / max(np.linalg.norm(num), 1e-30)
         assert rel <= 1e-6, (name, rel)
         np.testing.assert_allclose(ana, num, rtol=1e-5, atol=1e-7)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_row_dq_matches_finite_differences(causal):
+    # dQ of a subset of rows, straight from the finite differences of the
+    # brute-force forward (row i of dQ only moves O_i)
+    r = _rng(210 + causal)
+    n, d = 9, 3
+    q, k, v, do = (r.standard_normal((n, d)) for _ in range(4))
+    rows = np.array([0, 4, 8])
+    dq_rows = attn_dq_rows_ref(q, k, v, do, 0.7, causal, rows=rows)
+    num = _fd_grads(q, k, v, do, 0.7, causal)[0]
+    np.testing.assert_allclose(dq_rows, num[rows], rtol=1e-5, atol=1e-7)
+
+
+def test_row_dq_with_stored_o():
+    # an identity "storage" gives the exact gradient; a perturbed O changes dQ
+    # by exactly -scale * dD_i * (P K)_i, the only term in which D appears
+    r = _rng(212)
+    n, d = 11, 4
+    q, k, v, do = (r.standard_normal((n, d)) for _ in range(4))
+    rows = np.arange(n)
+    exact, same, shifted = attn_dq_rows_ref(q, k, v, do, 0.5, True, rows=rows,
+                                            o_for_d=[None, lambda o: o, lambda o: o + 0.01])
+    np.testing.assert_array_equal(same, exact)
+    p = attn_probs_ref(q, k, 0.5, True)
+    d_d = (do * 0.01).sum(-1, keepdims=True)
+    np.testing.assert_allclose(shifted - exact, -0.5 * d_d * (p @ k), rtol=1e-10, atol=1e-13)
 
 
 @pytest.mark.parametrize("causal", [False, True])
