@@ -37,7 +37,6 @@ __all__ = [
     "fa_last_device_status",
     "fa_debug_set_wait_limit_ms",
     "fa_debug_set_flags",
-    "fa_debug_exp2_poly",
     "fa_version",
     "FA_OK",
     "FA_ERR_INVALID_ARG",
@@ -93,7 +92,6 @@ _SIGNATURES = {
     "fa_last_device_status": (_c_int, [_vp]),
     "fa_debug_set_wait_limit_ms": (_c_int, [_c_int]),
     "fa_debug_set_flags": (_c_int, [_c_int]),
-    "fa_debug_exp2_poly": (_c_int, [_vp, _vp, _c_int, _vp]),
     "fa_version": (ctypes.c_char_p, []),
 }
 EXPORTED_SYMBOLS = tuple(_SIGNATURES)
@@ -170,28 +168,42 @@ def fa_debug_set_flags(flags: int) -> int:
     return load_library().fa_debug_set_flags(int(flags))
 
 
-def fa_debug_exp2_poly(x, stream=None):
-    """2^x by the library's FMA-pipe polynomial (diagnostics); x: CUDA float32."""
-    torch = _torch()
-    if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
-        raise ValueError("x must be a contiguous CUDA float32 tensor")
-    y = torch.empty_like(x)
-    st = load_library().fa_debug_exp2_poly(x.data_ptr(), y.data_ptr(), x.numel(), _stream_handle(stream))
-    if st != FA_OK:
-        raise FAError(st, "fa_debug_exp2_poly")
-    return y
-
-
 def _torch():
     import torch
     return torch
 
 
-def _stream_handle(stream) -> Optional[int]:
+def _stream_handle(stream, device=None) -> Optional[int]:
+    """Raw cudaStream_t of ``stream``; None means the current stream of
+    ``device`` (the device the call's tensors live on)."""
     torch = _torch()
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _on(t):
+    """Context that makes the device of tensor ``t`` current for a library
+    call: the library launches on the current device, resolves its status word
+    (and the fixed scratch of fa_bwd_noalloc) there, and every pointer it is
+    given must belong to that device."""
+    return _torch().cuda.device(t.device)
+
+
+def _check_workspace(ws, q):
+    if not getattr(ws, "is_cuda", False) or ws.device != q.device or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor on q's device")
+
+
+def _check_lse(lse, q):
+    """lse must be a contiguous float32 [B, H, N] CUDA tensor on q's device."""
+    B, H, N = q.shape[0], q.shape[1], q.shape[2]
+    if not getattr(lse, "is_cuda", False):
+        raise ValueError("lse must be a CUDA tensor (a host pointer would reach the kernels)")
+    if lse.device != q.device:
+        raise ValueError(f"lse is on {lse.device}, q on {q.device}: they must share a device")
+    if tuple(lse.shape) != (B, H, N) or lse.dtype != _torch().float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B, H, N] tensor")
 
 
 def fa_last_device_status(stream=None) -> int:
@@ -244,11 +256,12 @@ def fa_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: boo
         _check_bhnd("o", o, q, allow_f32=True)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    elif lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous float32 [B, H, N] tensor")
-    st = load_library().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                               B, H, N, d, float(scale), int(bool(causal)), _dtype_code(q, o),
-                               _stream_handle(stream))
+    else:
+        _check_lse(lse, q)
+    with _on(q):
+        st = load_library().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                   B, H, N, d, float(scale), int(bool(causal)), _dtype_code(q, o),
+                                   _stream_handle(stream, q.device))
     if st != FA_OK:
         raise FAError(st, "fa_fwd")
     return o, lse
@@ -265,8 +278,7 @@ def fa_bwd(q, k, v, o, do, lse, dq=None, dk=None, dv=None, workspace=None,
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
         _check_bhnd(name, t, None if name == "q" else q, allow_f32=(name == "o"))
     B, H, N, d = q.shape
-    if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous float32 [B, H, N] tensor")
+    _check_lse(lse, q)
     if scale is None:
         scale = 1.0 / float(d) ** 0.5
     dq = torch.empty_like(q) if dq is None else dq
@@ -277,11 +289,14 @@ def fa_bwd(q, k, v, o, do, lse, dq=None, dk=None, dv=None, workspace=None,
     need = fa_bwd_workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    st = load_library().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
-                               lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                               workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                               B, H, N, d, float(scale), int(bool(causal)), _dtype_code(q, o),
-                               _stream_handle(stream))
+    else:
+        _check_workspace(workspace, q)
+    with _on(q):
+        st = load_library().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                   lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                   workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                   B, H, N, d, float(scale), int(bool(causal)), _dtype_code(q, o),
+                                   _stream_handle(stream, q.device))
     if st != FA_OK:
         raise FAError(st, "fa_bwd")
     return dq, dk, dv
@@ -296,8 +311,7 @@ def fa_bwd_noalloc(q, k, v, o, do, lse, dq=None, dk=None, dv=None, scale: Option
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
         _check_bhnd(name, t, None if name == "q" else q, allow_f32=(name == "o"))
     B, H, N, d = q.shape
-    if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous float32 [B, H, N] tensor")
+    _check_lse(lse, q)
     if scale is None:
         scale = 1.0 / float(d) ** 0.5
     dq = torch.empty_like(q) if dq is None else dq
@@ -305,10 +319,11 @@ def fa_bwd_noalloc(q, k, v, o, do, lse, dq=None, dk=None, dv=None, scale: Option
     dv = torch.empty_like(q) if dv is None else dv
     for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
         _check_bhnd(name, t, q)
-    st = load_library().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
-                                       lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                                       B, H, N, d, float(scale), int(bool(causal)), _dtype_code(q, o),
-                                       _stream_handle(stream))
+    with _on(q):
+        st = load_library().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                           lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                           B, H, N, d, float(scale), int(bool(causal)), _dtype_code(q, o),
+                                           _stream_handle(stream, q.device))
     if st != FA_OK:
         raise FAError(st, "fa_bwd_noalloc")
     return dq, dk, dv
@@ -341,11 +356,12 @@ def fa_fwd_gqa(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal:
         _check_bhnd("o", o, q, allow_f32=True)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    elif lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous float32 [B, H, N] tensor")
-    st = load_library().fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                                   B, H, Hkv, N, d, float(scale), int(bool(causal)), _dtype_code(q, o),
-                                   _stream_handle(stream))
+    else:
+        _check_lse(lse, q)
+    with _on(q):
+        st = load_library().fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                       B, H, Hkv, N, d, float(scale), int(bool(causal)), _dtype_code(q, o),
+                                       _stream_handle(stream, q.device))
     if st != FA_OK:
         raise FAError(st, "fa_fwd_gqa")
     return o, lse
@@ -362,8 +378,7 @@ def fa_bwd_gqa(q, k, v, o, do, lse, dq=None, dk=None, dv=None, workspace=None,
     _check_bhnd("do", do, q)
     B, H, N, d = q.shape
     Hkv = k.shape[1]
-    if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous float32 [B, H, N] tensor")
+    _check_lse(lse, q)
     if scale is None:
         scale = 1.0 / float(d) ** 0.5
     dq = torch.empty_like(q) if dq is None else dq
@@ -375,11 +390,14 @@ def fa_bwd_gqa(q, k, v, o, do, lse, dq=None, dk=None, dv=None, workspace=None,
     need = fa_bwd_workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    st = load_library().fa_bwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
-                                   lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                                   workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                                   B, H, Hkv, N, d, float(scale), int(bool(causal)), _dtype_code(q, o),
-                                   _stream_handle(stream))
+    else:
+        _check_workspace(workspace, q)
+    with _on(q):
+        st = load_library().fa_bwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                       lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                       workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                       B, H, Hkv, N, d, float(scale), int(bool(causal)), _dtype_code(q, o),
+                                       _stream_handle(stream, q.device))
     if st != FA_OK:
         raise FAError(st, "fa_bwd_gqa")
     return dq, dk, dv
@@ -391,6 +409,8 @@ def _check_mask(block_mask, q):
     nb = (N + 127) // 128
     if not block_mask.is_cuda or block_mask.dtype != torch.uint8 or not block_mask.is_contiguous():
         raise ValueError("block_mask must be a contiguous CUDA uint8 tensor")
+    if block_mask.device != q.device:
+        raise ValueError("block_mask must be on q's device")
     if tuple(block_mask.shape[-2:]) != (nb, nb):
         raise ValueError(f"block_mask must end in ({nb}, {nb}) for N = {N}")
     if block_mask.dim() == 2:
@@ -418,9 +438,12 @@ def fa_fwd_blocksparse(q, k, v, block_mask, o=None, lse=None, scale: Optional[fl
         _check_bhnd("o", o, q, allow_f32=True)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    st = load_library().fa_fwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+    else:
+        _check_lse(lse, q)
+    with _on(q):
+        st = load_library().fa_fwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                                            block_mask.data_ptr(), stride, B, H, N, d, float(scale),
-                                           int(bool(causal)), _dtype_code(q, o), _stream_handle(stream))
+                                           int(bool(causal)), _dtype_code(q, o), _stream_handle(stream, q.device))
     if st != FA_OK:
         raise FAError(st, "fa_fwd_blocksparse")
     return o, lse
@@ -442,20 +465,24 @@ def fa_bwd_blocksparse(q, k, v, o, do, lse, block_mask, dq=None, dk=None, dv=Non
     need = fa_bwd_workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    st = load_library().fa_bwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
-                                           lse.data_ptr(), block_mask.data_ptr(), stride, dq.data_ptr(),
-                                           dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
-                                           workspace.numel() * workspace.element_size(), B, H, N, d, float(scale),
-                                           int(bool(causal)), _dtype_code(q, o), _stream_handle(stream))
+    else:
+        _check_workspace(workspace, q)
+    with _on(q):
+        st = load_library().fa_bwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                               lse.data_ptr(), block_mask.data_ptr(), stride, dq.data_ptr(),
+                                               dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                                               workspace.numel() * workspace.element_size(), B, H, N, d, float(scale),
+                                               int(bool(causal)), _dtype_code(q, o), _stream_handle(stream, q.device))
     if st != FA_OK:
         raise FAError(st, "fa_bwd_blocksparse")
     return dq, dk, dv
 
 
-def _dense_cuda(name, t, dtypes):
-    torch = _torch()
+def _dense_cuda(name, t, dtypes, ref=None):
     if not t.is_cuda or not t.is_contiguous() or t.dtype not in dtypes:
         raise ValueError(f"{name} must be a contiguous CUDA tensor of type {dtypes}")
+    if ref is not None and t.device != ref.device:
+        raise ValueError(f"{name} must be on the same device as the other arguments")
 
 
 def fa_merge(o, lse, o_part, lse_part, out=None, stream=None):
@@ -464,21 +491,22 @@ def fa_merge(o, lse, o_part, lse_part, out=None, stream=None):
     (optional, bf16/fp16, shape of o) receives the merged O as well."""
     torch = _torch()
     for name, t in (("o", o), ("o_part", o_part)):
-        _dense_cuda(name, t, (torch.float32,))
+        _dense_cuda(name, t, (torch.float32,), o)
     for name, t in (("lse", lse), ("lse_part", lse_part)):
-        _dense_cuda(name, t, (torch.float32,))
+        _dense_cuda(name, t, (torch.float32,), o)
     if o_part.shape != o.shape or lse.shape != o.shape[:-1] or lse_part.shape != lse.shape:
         raise ValueError("fa_merge: shapes of o, o_part, lse, lse_part disagree")
     code = -1
     if out is not None:
-        _dense_cuda("out", out, (torch.bfloat16, torch.float16))
+        _dense_cuda("out", out, (torch.bfloat16, torch.float16), o)
         if out.shape != o.shape:
             raise ValueError("fa_merge: out must have the shape of o")
         code = FA_BF16 if out.dtype == torch.bfloat16 else FA_FP16
     d = o.shape[-1]
-    st = load_library().fa_merge(o.data_ptr(), lse.data_ptr(), o_part.data_ptr(), lse_part.data_ptr(),
-                                 out.data_ptr() if out is not None else None, code, lse.numel(), d,
-                                 _stream_handle(stream))
+    with _on(o):
+        st = load_library().fa_merge(o.data_ptr(), lse.data_ptr(), o_part.data_ptr(), lse_part.data_ptr(),
+                                     out.data_ptr() if out is not None else None, code, lse.numel(), d,
+                                     _stream_handle(stream, o.device))
     if st != FA_OK:
         raise FAError(st, "fa_merge")
     return o, lse
@@ -488,12 +516,13 @@ def fa_grad_accumulate(acc, src, stream=None):
     """In place: acc (fp32) += src (bf16/fp16), elementwise, same shape."""
     torch = _torch()
     _dense_cuda("acc", acc, (torch.float32,))
-    _dense_cuda("src", src, (torch.bfloat16, torch.float16))
+    _dense_cuda("src", src, (torch.bfloat16, torch.float16), acc)
     if acc.shape != src.shape:
         raise ValueError("fa_grad_accumulate: shapes differ")
-    st = load_library().fa_grad_accumulate(acc.data_ptr(), src.data_ptr(), acc.numel(),
-                                           FA_BF16 if src.dtype == torch.bfloat16 else FA_FP16,
-                                           _stream_handle(stream))
+    with _on(acc):
+        st = load_library().fa_grad_accumulate(acc.data_ptr(), src.data_ptr(), acc.numel(),
+                                               FA_BF16 if src.dtype == torch.bfloat16 else FA_FP16,
+                                               _stream_handle(stream, acc.device))
     if st != FA_OK:
         raise FAError(st, "fa_grad_accumulate")
     return acc
@@ -505,11 +534,12 @@ def fa_convert(src, dtype=None, out=None, stream=None):
     _dense_cuda("src", src, (torch.float32,))
     if out is None:
         out = torch.empty(src.shape, dtype=dtype or torch.bfloat16, device=src.device)
-    _dense_cuda("out", out, (torch.bfloat16, torch.float16))
+    _dense_cuda("out", out, (torch.bfloat16, torch.float16), src)
     if out.shape != src.shape:
         raise ValueError("fa_convert: shapes differ")
-    st = load_library().fa_convert(out.data_ptr(), src.data_ptr(), src.numel(),
-                                   FA_BF16 if out.dtype == torch.bfloat16 else FA_FP16, _stream_handle(stream))
+    with _on(src):
+        st = load_library().fa_convert(out.data_ptr(), src.data_ptr(), src.numel(),
+                                       FA_BF16 if out.dtype == torch.bfloat16 else FA_FP16, _stream_handle(stream, src.device))
     if st != FA_OK:
         raise FAError(st, "fa_convert")
     return out
@@ -547,9 +577,10 @@ def fa_fp8_quantize(q, k, v, signs=None, workspace=None, stream=None):
     B, H, N, d = q.shape
     if workspace is None:
         workspace = torch.empty(fa_fwd_fp8_workspace_size(B, H, N, d), dtype=torch.uint8, device=q.device)
-    st = load_library().fa_fp8_quantize(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                        signs.data_ptr() if signs is not None else None, workspace.data_ptr(),
-                                        workspace.numel(), B, H, N, d, _dtype_code(q, q), _stream_handle(stream))
+    with _on(q):
+        st = load_library().fa_fp8_quantize(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                            signs.data_ptr() if signs is not None else None, workspace.data_ptr(),
+                                            workspace.numel(), B, H, N, d, _dtype_code(q, q), _stream_handle(stream, q.device))
     if st != FA_OK:
         raise FAError(st, "fa_fp8_quantize")
     return _fp8_views(workspace, B, H, N)
@@ -563,8 +594,9 @@ def fa_fwd_fp8(q, k, v, signs=None, o=None, lse=None, workspace=None, scale: Opt
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check_bhnd(name, t, None if name == "q" else q)
     B, H, N, d = q.shape
-    if signs is not None and (not signs.is_cuda or signs.dtype != torch.float32 or signs.numel() != d):
-        raise ValueError("signs must be a CUDA float32 tensor of d entries")
+    if signs is not None and (not signs.is_cuda or signs.dtype != torch.float32 or signs.numel() != d
+                              or signs.device != q.device or not signs.is_contiguous()):
+        raise ValueError("signs must be a contiguous CUDA float32 tensor of d entries on q's device")
     if scale is None:
         scale = 1.0 / float(d) ** 0.5
     if o is None:
@@ -573,10 +605,11 @@ def fa_fwd_fp8(q, k, v, signs=None, o=None, lse=None, workspace=None, scale: Opt
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     if workspace is None:
         workspace = torch.empty(max(1, fa_fwd_fp8_workspace_size(B, H, N, d)), dtype=torch.uint8, device=q.device)
-    st = load_library().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                                   signs.data_ptr() if signs is not None else None, workspace.data_ptr(),
-                                   workspace.numel(), B, H, N, d, float(scale), int(bool(causal)),
-                                   _dtype_code(q, o), _stream_handle(stream))
+    with _on(q):
+        st = load_library().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                       signs.data_ptr() if signs is not None else None, workspace.data_ptr(),
+                                       workspace.numel(), B, H, N, d, float(scale), int(bool(causal)),
+                                       _dtype_code(q, o), _stream_handle(stream, q.device))
     if st != FA_OK:
         raise FAError(st, "fa_fwd_fp8")
     return o, lse

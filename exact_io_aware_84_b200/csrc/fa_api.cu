@@ -153,11 +153,6 @@ int check_common(int B, int H, int N, int d, float scale, int dtype) {
   return FA_OK;
 }
 
-__global__ void exp2_poly_kernel(const float* x, float* y, int n) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) y[i] = exp2_poly(x[i]);
-}
-
 uint64_t wait_limit_ns() { return (uint64_t)g_wait_limit_ms.load() * 1000000ull; }
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -203,15 +198,6 @@ int fa_last_device_status(void* stream) {
   if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
   if (v != 0 && cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
   return v;
-}
-
-int fa_debug_exp2_poly(const float* x, float* y, int n, void* stream) {
-  if (!x || !y || n <= 0) return FA_ERR_INVALID_ARG;
-  DeviceInfo di;
-  int st = device_info(&di);
-  if (st != FA_OK) return st;
-  exp2_poly_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,

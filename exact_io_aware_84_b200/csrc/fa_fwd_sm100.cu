@@ -33,25 +33,6 @@ constexpr int kFwdThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only if max grows > 2^8
-// Which of the 8 element pairs in every 16 columns take exp2 on the FMA pipe
-// (exp2_poly) instead of the MUFU unit: bit k set = pair k.  The MUFU alone
-// caps the softmax at 16 exponentials/clock/SM; at d = 64 each exponential
-// carries half the MMA work of d = 128, so only d = 64 is MUFU-bound.
-#ifndef FA_FWD_POLY_PAIR_MASK_D64
-#define FA_FWD_POLY_PAIR_MASK_D64 0x00
-#endif
-#ifndef FA_FWD_POLY_PAIR_MASK_D128
-#define FA_FWD_POLY_PAIR_MASK_D128 0x00
-#endif
-// The FP8 variant's products take half the time of the 16-bit ones, so its
-// softmax is MUFU-bound at d = 128 as well.
-#ifndef FA_FWD_POLY_PAIR_MASK_FP8
-#define FA_FWD_POLY_PAIR_MASK_FP8 0x00
-#endif
-template <int D, bool FP8 = false>
-constexpr uint32_t poly_pair_mask() {
-  return FP8 ? FA_FWD_POLY_PAIR_MASK_FP8 : D == 64 ? FA_FWD_POLY_PAIR_MASK_D64 : FA_FWD_POLY_PAIR_MASK_D128;
-}
 // Register split.  Launch: 384 threads x 168 registers.  Warp w runs on SM
 // sub-partition w % 4, which therefore holds warps {k, k+4, k+8}: two softmax
 // warps and one warp of the producer/MMA warpgroup.  Each sub-partition's
@@ -658,9 +639,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int e = 0; e < 16; ++e) {
             float x0, x1;
             f2_unpack(f2_fma(f2_pack(s[32 * q + 2 * e], s[32 * q + 2 * e + 1]), cl2x2, nm2), x0, x1);
-            const bool poly = (poly_pair_mask<D, FP8>() >> (e & 7)) & 1u;
-            const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
-            const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+            const float p0 = ex2_approx(x0);
+            const float p1 = ex2_approx(x1);
             ps2[e & 3] = f2_add(ps2[e & 3], f2_pack(p0, p1));
             if constexpr (FP8) {
               // two e4m3 per 16 bits; element pairs (2e, 2e + 1) of 32 keys

@@ -26,12 +26,24 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
 
+// Per-device address of the array.  Only a successful lookup is kept: a
+// first call that fails (made during stream capture, or with an earlier
+// error pending) leaves the slot empty and a later call tries again.
 struct DeviceScratch {
-  std::once_flag once;
+  std::mutex mu;
   void* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
 };
 DeviceScratch g_scratch[kMaxDevices];
+
+void* scratch_address(int dev) {
+  DeviceScratch& s = g_scratch[dev];
+  std::lock_guard<std::mutex> lock(s.mu);
+  if (s.ptr == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) == cudaSuccess) s.ptr = p;
+  }
+  return s.ptr;
+}
 
 }  // namespace
 
@@ -39,17 +51,21 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
                               const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                               float scale, int causal, int dtype, void* stream) {
   const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  if (need == 0 || !q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) {
+    // invalid arguments: fa_bwd reports which, before it would touch any
+    // workspace; the scratch is not looked up
+    return fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, nullptr, 0, B, H, N, d, scale, causal, dtype, stream);
+  }
   if (need > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;  // problem too large for the fixed scratch
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_NO_DEVICE;
-  DeviceScratch& s = g_scratch[dev];
-  // First call on this device (with it current): resolve the array's device
-  // address.  Make this first call before any stream capture.
-  std::call_once(s.once, [&s] { s.err = cudaGetSymbolAddress(&s.ptr, g_noalloc_scratch); });
-  if (s.err != cudaSuccess || s.ptr == nullptr) return FA_ERR_CUDA;
+  // The first successful call on a device (with it current) resolves the
+  // array's device address; make that first call before any stream capture.
+  void* ws = scratch_address(dev);
+  if (ws == nullptr) return FA_ERR_CUDA;
   // fa_bwd rewrites all of the scratch it reads (it zeroes the dQ accumulator
   // and recomputes the row vectors), so stale contents from an earlier call
   // do not matter.  Calls that overlap on the GPU share the array and race.
-  return fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, s.ptr, kNoAllocScratchBytes, B, H, N, d, scale, causal,
-                dtype, stream);
+  return fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, ws, kNoAllocScratchBytes, B, H, N, d, scale, causal, dtype,
+                stream);
 }

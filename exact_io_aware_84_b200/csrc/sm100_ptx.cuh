@@ -313,26 +313,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// Base-2 exponential on the FMA pipe, for inputs x <= 64 (the softmax only
-// passes x <= ~8).  Cody-Waite split x = j + f with j = rint(x) (the
-// 1.5 * 2^23 rounding constant) and f in [-0.5, 0.5]; 2^f by a degree-3
-// polynomial fitted for minimax relative error on [-0.5, 0.5] (max relative
-// error 7.5e-5, below the 2^-9 spacing of bf16); 2^j is added into the
-// exponent field.  Inputs below -125 (including -inf) are clamped to -125, so
-// every result stays a normal float (they return ~2e-38 instead of 0).  Used
-// for a fraction of the softmax exponentials to take load off the MUFU unit.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float kRound = 12582912.f;  // 1.5 * 2^23
-  const float t = x + kRound;       // j in the low mantissa bits (round to nearest)
-  const float j = t - kRound;
-  const float f = x - j;
-  float p = fmaf(0.055171579f, f, 0.24261102f);
-  p = fmaf(p, f, 0.69326097f);
-  p = fmaf(p, f, 0.99992806f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // Pack two fp32 into one 32-bit word of 16-bit floats: `lo` in bits 0-15.
 template <bool BF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {

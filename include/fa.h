@@ -130,8 +130,11 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
  *   that loads the library until the process exits.  Problems whose
  *   fa_bwd_workspace_size exceeds it return FA_ERR_WORKSPACE before anything
  *   runs.  The call allocates nothing.
- *   The first call on each device looks up the array's device address (with
- *   that device current); make that first call before any stream capture.
+ *   Invalid arguments are reported (as by fa_bwd) without touching the
+ *   array.  The first successful call on each device looks up the array's
+ *   device address (with that device current) and keeps it; a lookup that
+ *   fails returns FA_ERR_CUDA and is retried by the next call.  Make the
+ *   first call on a device before any stream capture.
  *   All calls on a device share the array: calls that overlap on the GPU
  *   (other streams, other host threads) race and must be serialised by the
  *   caller.  The array keeps the last call's contents; fa_bwd rewrites every
@@ -286,17 +289,6 @@ int fa_last_device_status(void* stream);
  */
 int fa_debug_set_wait_limit_ms(int ms);
 int fa_debug_set_flags(int flags);
-
-/*
- * Diagnostics: y[i] = 2^x[i] computed by the FMA-pipe polynomial the forward
- * kernel can use for part of its softmax exponentials (Cody-Waite split into
- * integer and fractional part, degree-3 minimax polynomial for 2^f on
- * [-0.5, 0.5], relative error < 1e-4 for -125 <= x <= 64; inputs below -125
- * are clamped to -125 and give about 2e-38).  x, y: device float arrays of n elements.  One launch on
- * `stream`.  Not part of the attention computation's interface; it exists so
- * that the polynomial can be checked against the hardware exponential.
- */
-int fa_debug_exp2_poly(const float* x, float* y, int n, void* stream);
 
 /* Version string of the library build. */
 const char* fa_version(void);

@@ -57,3 +57,22 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     p = ctypes.c_void_p(0x1000)
     st = lib.fa_bwd_noalloc(p, p, p, p, p, p, p, p, p, 4, 16, 16384, 128, ctypes.c_float(0.1), 0, 0, None)
     assert st == fa.FA_ERR_WORKSPACE
+
+
+def test_noalloc_through_the_python_wrapper():
+    # the same entry point through the binding (argument checks, device
+    # context, stream of q's device), against fa_bwd on the same inputs
+    w = Workload("noalloc_wrap", 1, 2, 300, 64, "bf16", True, 0.125, True, seed=23)
+    x = make_inputs(w)
+    g = {k: v.cuda() for k, v in x.items()}
+    o, lse = fa.fa_fwd(g["q"], g["k"], g["v"], scale=w.scale, causal=w.causal)
+    ref = fa.fa_bwd(g["q"], g["k"], g["v"], o, g["do"], lse, scale=w.scale, causal=w.causal)
+    for _ in range(2):
+        got = fa.fa_bwd_noalloc(g["q"], g["k"], g["v"], o, g["do"], lse, scale=w.scale, causal=w.causal)
+        torch.cuda.synchronize()
+        assert fa.fa_last_device_status() == fa.FA_OK
+        for name, a, r in zip(("dq", "dk", "dv"), got, ref):
+            e = rel_fro(to64(a), to64(r))
+            assert e <= TOL_GRAD_REL, (name, e)
+    with pytest.raises(ValueError):
+        fa.fa_bwd_noalloc(g["q"], g["k"], g["v"], o, g["do"], lse.cpu(), scale=w.scale, causal=w.causal)
