@@ -2,9 +2,14 @@
 """Benchmark: attention forward + backward TFLOP/s on B200 through libfa.so.
 
 One step = the whole hot path over one batch: fa_fwd (O, LSE) then fa_bwd
-(dQ, dK, dV) on seeded synthetic inputs of the named workload.  FLOPs per
-step follow the pages' convention: 4 B H N^2 d for the forward (halved when
-causal) and 2.5x that for the backward.
+(dQ, dK, dV) on seeded synthetic inputs of the named workload (default: the
+d = 128, N = 8192, non-causal workload, B = 2, H = 16).  A step that has a
+backward is the training path: the forward stores O in float32 and the
+backward reads it for D = rowsum(dO o O) (bf16 storage of O alone puts the
+trading-day dQ over the 1e-2 tolerance).  FLOPs per step follow the pages'
+convention: 4 B H N^2 d for the forward (halved when causal) and 2.5x that
+for the backward.  The line also carries ``per_config``: forward and
+backward TFLOP/s of every workload, timed the same way.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the fp64 CPU oracle, timed as is
@@ -32,8 +37,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-DEFAULT_WORKLOAD = "gpt2_batch"  # B=8 H=12 N=1024 d=64 bf16 causal, forward + backward
-TARGET_WORKLOAD = "d128_n8192_nc"  # B=2 H=16 N=8192 d=128 bf16 non-causal
+DEFAULT_WORKLOAD = "d128_n8192_nc"  # B=2 H=16 N=8192 d=128 bf16 non-causal, forward + backward
+TARGET_WORKLOAD = "d128_n8192_nc"  # the >= 60%-of-peak forward criterion is quoted on this one
+PER_CONFIG = ("tiny_fwd", "gpt2_batch", "seq4k_fp16", "trading_day",
+              "d128_n2048_nc", "d128_n2048_causal", "d128_n8192_nc", "d128_n8192_causal",
+              "d128_n16384_nc", "d128_n16384_causal")
+BWD_LAUNCHES = 3   # fa_bwd: preprocess, main, dQ conversion
 METRIC = "attention fwd/bwd TFLOP/s on 1 B200 (bf16); % of dense BF16 tensor peak"
 L2_FLUSH_BYTES = 256 << 20
 
@@ -49,6 +58,8 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-target", action="store_true")
     ap.add_argument("--no-memory", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--per-config-steps", type=int, default=5)
     ap.add_argument("--variant", default="dense", choices=["dense", "gqa", "blocksparse", "fp8", "ring"],
                     help="dense attention (default); grouped-query attention with H/4 key/value heads; "
                          "block-sparse attention with a seeded random 128x128 tile mask keeping half the tiles; "
@@ -158,29 +169,50 @@ def _max_over_ranks(x, world):
 
 # ------------------------------------------------------------------ oracle leg
 
-def _oracle_sample(w, budget_s, seed=0, passes=1):
-    """Time the fp64 oracle (forward + backward) on whole heads of the
-    workload until ~budget_s of CPU work or ``passes`` passes over its B*H
-    heads; returns (TFLOP/s, heads, seconds)."""
-    import numpy as np
-    from exact_io_aware_84_b200.inputs import make_inputs
+ORACLE_HEAD_FLOP_CAP = 2.0e10   # fp64 FLOPs of one timed oracle unit (about 1-2 s on 16 cores)
+
+
+def _oracle_unit(w):
+    """The unit the CPU oracle is timed on: one whole (b, h) head, or, when one
+    head's fp64 forward (+ backward) would exceed ORACLE_HEAD_FLOP_CAP, the
+    first n positions of a head (n a multiple of 128; the same computation on a
+    shorter sequence, whose FLOPs are counted at its own length)."""
     from exact_io_aware_84_b200.metrics import attn_bwd_flops, attn_fwd_flops
+
+    def flops(n):
+        return attn_fwd_flops(1, 1, n, w.d, w.causal) + (attn_bwd_flops(1, 1, n, w.d, w.causal) if w.backward else 0)
+
+    n = w.N
+    while n > 128 and flops(n) > ORACLE_HEAD_FLOP_CAP:
+        n = max(128, (int(n * 0.9) // 128) * 128)
+    return n, flops(n)
+
+
+def _oracle_sample(w, budget_s, seed=0, passes=1):
+    """Time the fp64 oracle (forward + backward) on units of the workload
+    (``_oracle_unit``) until ~budget_s of CPU work or ``passes`` passes over
+    its B*H heads; returns (TFLOP/s, units, seconds, unit length)."""
+    from exact_io_aware_84_b200.inputs import make_inputs
     from oracle import attn_bwd_ref, attn_fwd_ref
-    one = w.with_(B=1, H=1, seed=seed)
+    n, flops_unit = _oracle_unit(w)
+    one = w.with_(B=1, H=1, N=n, seed=seed)
     x = make_inputs(one, with_grad=w.backward)
-    q, k, v = (x[n][0, 0].double().numpy() for n in ("q", "k", "v"))
+    q, k, v = (x[name][0, 0].double().numpy() for name in ("q", "k", "v"))
     do = x["do"][0, 0].double().numpy() if w.backward else None
-    flops_head = attn_fwd_flops(1, 1, w.N, w.d, w.causal) + (attn_bwd_flops(1, 1, w.N, w.d, w.causal) if w.backward else 0)
-    heads, t0 = 0, time.perf_counter()
+    units, t0 = 0, time.perf_counter()
     while True:
         attn_fwd_ref(q, k, v, w.scale, w.causal)
         if w.backward:
             attn_bwd_ref(q, k, v, do, w.scale, w.causal)
-        heads += 1
+        units += 1
         el = time.perf_counter() - t0
-        if el >= budget_s or heads >= passes * w.B * w.H:
+        if el >= budget_s or units >= passes * w.B * w.H:
             break
-    return flops_head * heads / el / 1e12, heads, el
+    return flops_unit * units / el / 1e12, units, el, n
+
+
+def _unit_words(w, n):
+    return "whole (b,h) heads" if n == w.N else f"(b,h) heads cut to their first {n} of {w.N} positions"
 
 
 def _cpu_threads():
@@ -204,9 +236,9 @@ def run_reference(args):
     per_step_budget = max(0.5, 150.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         _oracle_sample(w, per_step_budget / 4)
-    vals, secs, heads = [], 0.0, 0
+    vals, secs, heads, n = [], 0.0, 0, w.N
     for _ in range(args.steps):
-        v, h, el = _oracle_sample(w, per_step_budget)
+        v, h, el, n = _oracle_sample(w, per_step_budget)
         vals.append(v)
         secs += el
         heads += h
@@ -218,7 +250,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": _config(w, world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{heads} whole (b,h) heads of {w.name} (fp64 forward"
+                         "sample": f"{heads} {_unit_words(w, n)} of {w.name} (fp64 forward"
                                    f"{' + backward' if w.backward else ''}) over {args.steps} steps"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -249,7 +281,9 @@ def run_native(args):
     x = make_inputs(w.with_(seed=w.seed + rank), with_grad=w.backward)
     g = {k: v.to(dev) for k, v in x.items()}
     B, H, N, d = w.B, w.H, w.N, w.d
-    o = torch.empty_like(g["q"])
+    # the training path stores O in float32 for the backward's D term
+    o_fp32 = w.backward and args.variant in ("dense", "gqa", "blocksparse")
+    o = torch.empty(g["q"].shape, dtype=torch.float32 if o_fp32 else g["q"].dtype, device=dev)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     if w.backward:
         dq, dk, dv = (torch.empty_like(g["q"]) for _ in range(3))
@@ -257,7 +291,7 @@ def run_native(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     f_fwd = attn_fwd_flops(B, H, N, d, w.causal)
-    variant = {"name": args.variant}
+    variant = {"name": args.variant, "o_storage": "float32" if o_fp32 else w.dtype}
 
     if args.variant == "dense":
         def step():
@@ -368,17 +402,17 @@ def run_native(args):
                                       scale=w.scale, causal=w.causal, stream=stream)
 
     with_bwd = w.backward and args.variant != "fp8"
-    launches_per_step = (4 if args.variant == "fp8" else 1) + (3 if with_bwd else 0)
+    launches_per_step = (4 if args.variant == "fp8" else 1) + (BWD_LAUNCHES if with_bwd else 0)
     if args.variant == "ring":
         # per rank and step: forward 1 (+1 merge), backward 3 + 3 accumulates;
         # per rank: 1 + 3 conversions (skipped chunk pairs launch nothing);
         # counted for all emulated ranks on one GPU, for this rank with NCCL
         R = args.ring_size if world == 1 else world
         pairs = R * (R + 1) // 2 if w.causal else R * R
-        launches_per_step = (pairs + (pairs - R) + R) + ((6 * pairs + 3 * R) if with_bwd else 0)
+        launches_per_step = (pairs + (pairs - R) + R) + (((BWD_LAUNCHES + 3) * pairs + 3 * R) if with_bwd else 0)
         if world > 1:  # this rank's own launches (rank 0 prints)
             pr = rank + 1 if w.causal else world
-            launches_per_step = (2 * pr) + ((6 * pr + 3) if with_bwd else 0)
+            launches_per_step = (2 * pr) + (((BWD_LAUNCHES + 3) * pr + 3) if with_bwd else 0)
     f_bwd = 2.5 * f_fwd if with_bwd else 0.0
     flops = f_fwd + f_bwd
 
@@ -390,19 +424,24 @@ def run_native(args):
     if fa.fa_last_device_status(stream) != fa.FA_OK:
         raise RuntimeError("device status not OK after warm-up")
 
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    starts, mids, ends = (_events(torch, args.steps, stream) for _ in range(3))
+    # the backward's main kernel, bracketed by events the library records
+    # around its launch (dense / GQA / block-sparse backward)
+    time_main = with_bwd and args.variant in ("dense", "gqa", "blocksparse")
+    kb, ka = (_events(torch, args.steps, stream) for _ in range(2))
     _barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         for i in range(args.steps):
             flush.zero_()
+            if time_main:
+                fa.fa_debug_set_timing_events(kb[i], ka[i])
             starts[i].record(stream)
             ev_mid = mids[i]
             step()
             ends[i].record(stream)
         torch.cuda.synchronize()
+    fa.fa_debug_set_timing_events(None, None)
     _barrier(world)
     status = fa.fa_last_device_status(stream)
     if status != fa.FA_OK:
@@ -410,26 +449,38 @@ def run_native(args):
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     fwd_ms = [s.elapsed_time(m) for s, m in zip(starts, mids)]
     bwd_ms = [m.elapsed_time(e) for m, e in zip(mids, ends)]
+    main_ms = [b_.elapsed_time(a_) for b_, a_ in zip(kb, ka)] if time_main else None
     total_ms = _max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
     value = flops * world / (ms_per_step * 1e-3) / 1e12
     clocks = clk.summary()
 
-    # dominant kernel (the backward launch group when present, else the forward)
+    # dominant kernel: the backward's main kernel when there is a backward
+    # (timed live by the events the library records around its launch), else
+    # the forward kernel (the only launch between the step's first events)
     peaks = _peaks()
     # FP8 products run at twice the 16-bit rate (the recipe's nominal 4.5 vs
     # 2.25 PFLOP/s): their peak is the measured bf16 peak times 2
     dt_ratio = 2.0 if args.variant == "fp8" else 1.0
-    if with_bwd:
-        dom_ms, dom_flops, dom_name = statistics.mean(bwd_ms), f_bwd, "fa_bwd (prep + main + dQ convert launches)"
+    if time_main:
+        dom_ms, dom_flops, dom_name = statistics.mean(main_ms), f_bwd, "fa_bwd_main"
+        dom_how = ("backward FLOPs (2.5 x 4 B H N^2 d, x1/2 causal) / mean duration of fa_bwd_main, between "
+                   "CUDA events the library records on the launching stream right before and after its launch, "
+                   "in every timed step")
+    elif with_bwd:
+        dom_ms, dom_flops, dom_name = statistics.mean(bwd_ms), f_bwd, "fa_bwd (all launches)"
+        dom_how = "backward FLOPs / mean duration of the backward's launches (CUDA events around the call)"
     else:
-        dom_ms, dom_flops, dom_name = statistics.mean(fwd_ms), f_fwd, \
-            "fa_fwd_fp8 (quantise + fa_fwd_kernel FP8)" if args.variant == "fp8" else "fa_fwd_kernel"
+        dom_ms, dom_flops = statistics.mean(fwd_ms), f_fwd
+        dom_name = "fa_fwd_fp8 (quantise + fa_fwd_kernel FP8)" if args.variant == "fp8" else "fa_fwd_kernel"
+        dom_how = "forward FLOPs (4 B H N^2 d, x1/2 causal) / mean duration of the forward (CUDA events)"
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"] * dt_ratio
     roofline = {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak,
                 "traffic": _ncu_traffic(w.name, dom_name) if args.variant == "dense" else None,
+                "traffic_unit": "DRAM bytes per launch (ncu, current kernel sources only)",
+                "how": dom_how, "kernel_ms": dom_ms,
                 "peak_source": f"{peaks['source']} bf16 burst" + (" x 2 (fp8 / bf16 nominal)" if dt_ratio != 1 else ""),
                 "frac_of_sustained": achieved / (peaks["bf16_tflops_sustained"] * dt_ratio),
                 "fwd_tflops": f_fwd / (statistics.mean(fwd_ms) * 1e-3) / 1e12,
@@ -438,7 +489,7 @@ def run_native(args):
     # end to end through the public API: pinned host inputs -> device -> step -> host
     e2e = None
     if not args.no_e2e and args.variant == "dense":
-        e2e = _e2e(fa, torch, w, x, dev, stream, flops, world, args)
+        e2e = _e2e(fa, torch, w, x, dev, stream, flops, world, args, o_fp32=o_fp32)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -457,15 +508,17 @@ def run_native(args):
         "note": "the pages' own figures on other hardware; not targets",
         "fa2_a100_frac_of_peak": 0.70, "fa1_a100_frac_of_peak": 0.35,
         "source": "marketmaker.cc, FA2 section (A100 theoretical peak FLOPs)"}
-    if not args.no_target and w.name != TARGET_WORKLOAD and args.variant == "dense":
+    if not args.no_target and args.variant == "dense":
         line["target_fwd_d128_n8192_nc"] = _target_fwd(fa, torch, dev, stream, flush, peaks, args)
+    if not args.no_per_config and args.variant == "dense" and rank == 0:
+        line["per_config"] = _per_config(fa, torch, dev, stream, flush, peaks, args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.variant == "dense":
         # about 12 s of CPU work: a fraction of one pass over the heads of a
         # large workload, repeated passes over a small one
-        tf, heads, el = _oracle_sample(w, 12.0, passes=1000)
+        tf, heads, el, n_unit = _oracle_sample(w, 12.0, passes=1000)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": _cpu_threads(), "kind": "oracle",
-                                "sample": f"{heads} whole (b,h) heads ({heads / (w.B * w.H):.2f} passes over "
-                                          f"the {w.B * w.H} heads) of {w.name}, fp64 forward"
+                                "sample": f"{heads} {_unit_words(w, n_unit)} ({heads / (w.B * w.H):.2f} x the "
+                                          f"{w.B * w.H} heads) of {w.name}, fp64 forward"
                                           f"{' + backward' if w.backward else ''}, {el:.1f} s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -473,6 +526,80 @@ def run_native(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def _events(torch, n, stream):
+    """n timing events, each recorded once so that it exists before the
+    library is handed its handle."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for e in evs:
+        e.record(stream)
+    return evs
+
+
+def _per_config(fa, torch, dev, stream, flush, peaks, args):
+    """Forward and backward TFLOP/s of every workload, timed like the main leg
+    (CUDA events on the launching stream, L2 flushed before every step,
+    warm-up first): ``--per-config-steps`` timed steps after 3 warm-ups.  A
+    workload with a backward runs the training path (float32 O); its row also
+    carries the main backward kernel alone."""
+    from exact_io_aware_84_b200.inputs import make_inputs, workload
+    from exact_io_aware_84_b200.metrics import attn_bwd_flops, attn_fwd_flops
+    rows = {}
+    for name in PER_CONFIG:
+        w = workload(name)
+        x = make_inputs(w, with_grad=w.backward)
+        g = {k: v.to(dev) for k, v in x.items()}
+        B, H, N, d = w.B, w.H, w.N, w.d
+        o = torch.empty(g["q"].shape, dtype=torch.float32 if w.backward else g["q"].dtype, device=dev)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        if w.backward:
+            dq, dk, dv = (torch.empty_like(g["q"]) for _ in range(3))
+            ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+        n = max(1, args.per_config_steps)
+        ev = {k_: _events(torch, n, stream) for k_ in ("s", "m", "e", "kb", "ka")}
+
+        def step(i):
+            flush.zero_()
+            ev["s"][i].record(stream)
+            fa.fa_fwd(g["q"], g["k"], g["v"], o, lse, scale=w.scale, causal=w.causal, stream=stream)
+            ev["m"][i].record(stream)
+            if w.backward:
+                fa.fa_debug_set_timing_events(ev["kb"][i], ev["ka"][i])
+                fa.fa_bwd(g["q"], g["k"], g["v"], o, g["do"], lse, dq, dk, dv, ws, scale=w.scale,
+                          causal=w.causal, stream=stream)
+                fa.fa_debug_set_timing_events(None, None)
+            ev["e"][i].record(stream)
+
+        for _ in range(3):
+            step(0)
+        torch.cuda.synchronize()
+        for i in range(n):
+            step(i)
+        torch.cuda.synchronize()
+        if fa.fa_last_device_status(stream) != fa.FA_OK:
+            raise RuntimeError(f"device status not OK on {name}")
+        f_f = attn_fwd_flops(B, H, N, d, w.causal)
+        fwd_ms = statistics.mean(ev["s"][i].elapsed_time(ev["m"][i]) for i in range(n))
+        r = {"B": B, "H": H, "N": N, "d": d, "causal": w.causal, "dtype": w.dtype,
+             "o_storage": "float32" if w.backward else w.dtype, "steps": n,
+             "fwd_ms": fwd_ms, "fwd_tflops": f_f / (fwd_ms * 1e-3) / 1e12}
+        r["fwd_frac"] = r["fwd_tflops"] / peaks["bf16_tflops"]
+        if w.backward:
+            f_b = attn_bwd_flops(B, H, N, d, w.causal)
+            bwd_ms = statistics.mean(ev["m"][i].elapsed_time(ev["e"][i]) for i in range(n))
+            main_ms = statistics.mean(ev["kb"][i].elapsed_time(ev["ka"][i]) for i in range(n))
+            r.update(bwd_ms=bwd_ms, bwd_tflops=f_b / (bwd_ms * 1e-3) / 1e12,
+                     bwd_main_ms=main_ms, bwd_main_tflops=f_b / (main_ms * 1e-3) / 1e12,
+                     step_tflops=(f_f + f_b) / ((fwd_ms + bwd_ms) * 1e-3) / 1e12)
+            r["bwd_frac"] = r["bwd_tflops"] / peaks["bf16_tflops"]
+            r["bwd_main_frac"] = r["bwd_main_tflops"] / peaks["bf16_tflops"]
+        rows[name] = r
+        del g, o, lse, x
+        if w.backward:
+            del dq, dk, dv, ws
+        torch.cuda.empty_cache()
+    return rows
 
 
 def _attended_pairs(mask, N, causal):
@@ -557,7 +684,7 @@ def _target_fwd(fa, torch, dev, stream, flush, peaks, args):
             "target_frac": 0.60}
 
 
-def _e2e(fa, torch, w, x, dev, stream, flops, world, args, outputs=None):
+def _e2e(fa, torch, w, x, dev, stream, flops, world, args, outputs=None, o_fp32=False):
     """The metric end to end through the public calls: every step copies its
     inputs from pinned host memory to the device, runs fa_fwd (and fa_bwd)
     and copies all of its outputs (O, LSE, and dQ, dK, dV) back to pinned host
@@ -573,8 +700,8 @@ def _e2e(fa, torch, w, x, dev, stream, flops, world, args, outputs=None):
     out_names = ["o", "lse"] + (["dq", "dk", "dv"] if w.backward else [])
 
     def out_like(n, where):
-        if n == "lse":
-            t = torch.empty((B, H, N), dtype=torch.float32, device=where)
+        if n == "lse" or (n == "o" and o_fp32):
+            t = torch.empty((B, H, N) if n == "lse" else (B, H, N, d), dtype=torch.float32, device=where)
         else:
             t = torch.empty_like(pin["q"], device=where)
         return t.pin_memory() if where == "cpu" else t
@@ -677,21 +804,24 @@ def kernel_sources_hash():
     return h.hexdigest()[:16]
 
 
+TRAFFIC_RECORD = os.path.join("profiles", "traffic.json")
+
+
 def _ncu_traffic(workload_name, kernel_name):
-    """DRAM bytes per launch of the dominant kernel group, from the committed
-    ncu summary for this workload (profiles/traffic_<workload>.md), but only
-    while the kernel sources are the ones that summary was captured from;
-    otherwise null."""
-    import re
-    path = os.path.join(ROOT, "profiles", f"traffic_{workload_name}.md")
+    """DRAM bytes (read + write) per launch of ``kernel_name`` on the workload,
+    from the machine-readable record of the committed ncu capture
+    (profiles/traffic.json: {"kernel_sources": <hash>, "per_launch_bytes":
+    {workload: {kernel: bytes}}}), but only while the kernel sources are the
+    ones it was captured from; otherwise null."""
+    path = os.path.join(ROOT, TRAFFIC_RECORD)
     if not os.path.exists(path):
         return None
-    text = open(path).read()
-    m_hash = re.search(r"Kernel sources: `([0-9a-f]+)`", text)
-    m_val = re.search(r"bench\.py traffic key: " + re.escape(workload_name) + r"=(\d+)", text)
-    if not m_hash or not m_val or m_hash.group(1) != kernel_sources_hash():
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("kernel_sources") != kernel_sources_hash():
         return None
-    return int(m_val.group(1))
+    val = rec.get("per_launch_bytes", {}).get(workload_name, {}).get(kernel_name)
+    return int(val) if val is not None else None
 
 
 def main():

@@ -37,6 +37,7 @@ __all__ = [
     "fa_last_device_status",
     "fa_debug_set_wait_limit_ms",
     "fa_debug_set_flags",
+    "fa_debug_set_timing_events",
     "fa_version",
     "FA_OK",
     "FA_ERR_INVALID_ARG",
@@ -92,6 +93,7 @@ _SIGNATURES = {
     "fa_last_device_status": (_c_int, [_vp]),
     "fa_debug_set_wait_limit_ms": (_c_int, [_c_int]),
     "fa_debug_set_flags": (_c_int, [_c_int]),
+    "fa_debug_set_timing_events": (_c_int, [_vp, _vp]),
     "fa_version": (ctypes.c_char_p, []),
 }
 EXPORTED_SYMBOLS = tuple(_SIGNATURES)
@@ -166,6 +168,14 @@ def fa_debug_set_wait_limit_ms(ms: int) -> int:
 
 def fa_debug_set_flags(flags: int) -> int:
     return load_library().fa_debug_set_flags(int(flags))
+
+
+def fa_debug_set_timing_events(before_main=None, after_main=None) -> int:
+    """Have every backward call record these torch.cuda.Event objects (timing
+    enabled, already recorded once so that they exist) around the launch of
+    its main kernel; None, None clears the setting."""
+    h = lambda e: None if e is None else e.cuda_event
+    return load_library().fa_debug_set_timing_events(h(before_main), h(after_main))
 
 
 def _torch():

@@ -38,6 +38,9 @@ int* status_ptr() {
 
 std::atomic<int> g_wait_limit_ms{1000};
 std::atomic<int> g_debug_flags{0};
+// Events recorded around the backward's main kernel (fa_debug_set_timing_events).
+std::atomic<void*> g_ev_main_before{nullptr};
+std::atomic<void*> g_ev_main_after{nullptr};
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -192,6 +195,12 @@ int fa_debug_set_flags(int flags) {
   return FA_OK;
 }
 
+int fa_debug_set_timing_events(void* before_main, void* after_main) {
+  g_ev_main_before.store(before_main);
+  g_ev_main_after.store(after_main);
+  return FA_OK;
+}
+
 int fa_last_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
   int v = 0, zero = 0;
@@ -314,7 +323,10 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
       encode_tile_map(&tdo, dout, bh, N, d, bf16, q_rows) != FA_OK)
     return FA_ERR_CUDA;
   const int grid = p.n_units < di.sms ? p.n_units : di.sms;
-  cudaError_t e = launch_bwd(d, bf16, o32, causal != 0, tq, tk, tv, tdo, p, grid, static_cast<cudaStream_t>(stream));
+  const cudaEvent_t ev_main[2] = {static_cast<cudaEvent_t>(g_ev_main_before.load()),
+                                  static_cast<cudaEvent_t>(g_ev_main_after.load())};
+  cudaError_t e = launch_bwd(d, bf16, o32, causal != 0, tq, tk, tv, tdo, p, grid, static_cast<cudaStream_t>(stream),
+                             ev_main);
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

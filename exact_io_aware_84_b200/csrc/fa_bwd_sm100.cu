@@ -770,7 +770,8 @@ __global__ void __launch_bounds__(256) fa_bwd_dq(const BwdParams p) {
 
 template <int D, bool BF16, bool CAUSAL>
 cudaError_t launch_bwd_t(bool o32, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const CUtensorMap& tdo, const BwdParams& p, int grid, cudaStream_t st) {
+                         const CUtensorMap& tdo, const BwdParams& p, int grid, cudaStream_t st,
+                         cudaEvent_t const* ev_main) {
   {
     // row groups of 32 / (D / 8) rows per warp; a grid of up to 16 blocks of
     // 8 warps per SM strides over them
@@ -787,9 +788,11 @@ cudaError_t launch_bwd_t(bool o32, const CUtensorMap& tq, const CUtensorMap& tk,
     constexpr int smem = BwdLayout<D>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    if (ev_main && ev_main[0] && (e = cudaEventRecord(ev_main[0], st)) != cudaSuccess) return e;
     e = launch_chained(kern, dim3(grid), dim3(kBwdThreads), smem, st, tq, tk, tv, tdo, p);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    if (ev_main && ev_main[1] && (e = cudaEventRecord(ev_main[1], st)) != cudaSuccess) return e;
   }
   {
     const long long groups = (long long)p.bh * p.N * (D / 8);
@@ -805,9 +808,9 @@ int bwd_threads() { return kBwdThreads; }
 
 cudaError_t launch_bwd(int d, bool bf16, bool o32, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p, int grid,
-                       cudaStream_t st) {
+                       cudaStream_t st, cudaEvent_t const* ev_main) {
 #define FA_BWD_CASE(DD, BB, CC) \
-  if (d == DD && bf16 == BB && causal == CC) return launch_bwd_t<DD, BB, CC>(o32, tq, tk, tv, tdo, p, grid, st);
+  if (d == DD && bf16 == BB && causal == CC) return launch_bwd_t<DD, BB, CC>(o32, tq, tk, tv, tdo, p, grid, st, ev_main);
   FA_BWD_CASE(64, true, false)
   FA_BWD_CASE(64, true, true)
   FA_BWD_CASE(64, false, false)

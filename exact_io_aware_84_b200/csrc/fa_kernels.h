@@ -119,9 +119,11 @@ cudaError_t launch_fp8_prep(bool bf16, const void* q, const void* k, const void*
                             const Fp8Buffers& b, int bh, int N, cudaStream_t st);
 int fwd_fp8_smem();
 
+// ev_main[0] / ev_main[1] (may be null): events recorded on `st` right
+// before and right after the launch of the main backward kernel.
 cudaError_t launch_bwd(int d, bool bf16, bool o32, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p, int grid,
-                       cudaStream_t st);
+                       cudaStream_t st, cudaEvent_t const* ev_main);
 
 // Ring-attention helpers (fa_ring.cu).  out_kind: 0 none, 1 bf16, 2 fp16.
 cudaError_t launch_merge(int d, int out_kind, float* o, float* lse, const float* o_part, const float* lse_part,

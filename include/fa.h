@@ -68,6 +68,10 @@ typedef enum {
  * about 1e-2 relative.  The *_O_F32 codes keep O in float32 (the forward's
  * own accumulator, normalised) so that D carries only the forward's
  * arithmetic error; they cost 2 extra bytes per element of O traffic.
+ * A caller that runs the backward (training) should store O this way: on
+ * the one-trading-day workload (N = 23400, peaked rows) bf16 storage of O
+ * alone puts dQ at 1.03e-2 - 1.16e-2 relative error, with every other step
+ * exact, while float32 storage leaves about 2e-7.
  */
 typedef enum { FA_BF16 = 0, FA_FP16 = 1, FA_BF16_O_F32 = 2, FA_FP16_O_F32 = 3 } fa_dtype;
 
@@ -289,6 +293,19 @@ int fa_last_device_status(void* stream);
  */
 int fa_debug_set_wait_limit_ms(int ms);
 int fa_debug_set_flags(int flags);
+
+/*
+ * Diagnostics: kernel timing.  While set (non-NULL), every backward call
+ * records `before_main` on its stream right before it launches its main
+ * kernel (the dK/dV/dQ kernel) and `after_main` right after, so that the
+ * elapsed time between the two events is that kernel's duration.  Both are
+ * cudaEvent_t handles created by the caller with timing enabled; the caller
+ * owns them and must clear the setting (NULL, NULL) before destroying them.
+ * Process-wide; a recorded event changes the chaining of the backward's
+ * launches (the main kernel then starts after the event, not overlapped with
+ * the end of the preprocessing kernel).  Returns FA_OK.
+ */
+int fa_debug_set_timing_events(void* before_main, void* after_main);
 
 /* Version string of the library build. */
 const char* fa_version(void);

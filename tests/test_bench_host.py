@@ -60,12 +60,24 @@ def test_kernel_hash_ignores_comment_edits(tmp_path, monkeypatch):
 
 
 def test_traffic_key_only_while_kernels_unchanged(tmp_path, monkeypatch):
+    import json
     (tmp_path / "profiles").mkdir()
-    (tmp_path / "profiles" / "traffic_w.md").write_text(
-        "Kernel sources: `0123456789abcdef`.\n\nbench.py traffic key: w=4096\n")
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"kernel_sources": "0123456789abcdef", "per_launch_bytes": {"w": {"fa_bwd_main": 4096}}}))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setattr(bench, "kernel_sources_hash", lambda: "0123456789abcdef")
-    assert bench._ncu_traffic("w", "fa_bwd") == 4096
-    assert bench._ncu_traffic("other", "fa_bwd") is None
+    assert bench._ncu_traffic("w", "fa_bwd_main") == 4096
+    assert bench._ncu_traffic("w", "fa_fwd_kernel") is None
+    assert bench._ncu_traffic("other", "fa_bwd_main") is None
     monkeypatch.setattr(bench, "kernel_sources_hash", lambda: "fedcba9876543210")
-    assert bench._ncu_traffic("w", "fa_bwd") is None
+    assert bench._ncu_traffic("w", "fa_bwd_main") is None
+
+
+def test_oracle_unit_is_bounded():
+    from exact_io_aware_84_b200.inputs import workload
+    for name in ("gpt2_batch", "trading_day", "d128_n8192_nc", "d128_n16384_causal", "tiny_fwd"):
+        w = workload(name)
+        n, flops = bench._oracle_unit(w)
+        assert n % 128 == 0 or n == w.N
+        assert n <= w.N and flops <= bench.ORACLE_HEAD_FLOP_CAP
+    assert bench._oracle_unit(workload("gpt2_batch"))[0] == 1024   # small heads stay whole
