@@ -21,12 +21,14 @@
 //   d = 128: dQ_i^T = K_j^T dS^T  (M = 128 head dims, both operands MN-major)
 // Query tile BR = 128 rows for d = 64 and 64 rows for d = 128, so that
 // S^T | dP^T | dV | dK | dQ fit in the 512 tensor-memory columns (448 used).
-// Roles (384 threads):
+// Roles (512 threads):
 //   warps 0-7   two compute warpgroups (thread = key = TMEM lane), each owning
-//               half of every query tile's columns: P^T, the staging of the
-//               previous tile's dQ, dS^T; at the end of a unit each writes
-//               half of the head dims of dK and dV
-//   warp  8     TMA producer      warp 9   MMA issuer      warps 10-11 idle
+//               half of every query tile's columns: P^T, then dS^T; at the
+//               end of a unit each writes half of the head dims of dK and dV
+//   warps 8-11  dQ warpgroup: drains each query tile's dQ from tensor memory
+//               into shared memory and adds it into the fp32 accumulator
+//               with bulk reduce-adds, concurrently with the compute warps
+//   warp  12    TMA producer      warp 13  MMA issuer      warps 14-15 idle
 #include <cuda_fp16.h>
 
 #include <type_traits>
@@ -38,15 +40,19 @@ namespace fa {
 
 namespace {
 
-constexpr int kBwdThreads = 384;
-constexpr int kBProducerWarp = 8;
-constexpr int kBMmaWarp = 9;
-// Register split (same reasoning as the forward): every SM sub-partition holds
-// two warps of warpgroups 0-1 and one of warpgroup 2.
-constexpr int kBLaunchRegs = 168;
-constexpr int kBRegsWide = 192;
-constexpr int kBRegsNarrow = 120;
-static_assert(2 * kBRegsWide + kBRegsNarrow <= 3 * kBLaunchRegs, "register split exceeds a sub-partition's pool");
+constexpr int kBwdThreads = 512;
+constexpr int kBDqWarp0 = 8;         // warps 8-11: dQ warpgroup (TMEM lane quadrants 0-3)
+constexpr int kBProducerWarp = 12;
+constexpr int kBMmaWarp = 13;
+// Register split: every SM sub-partition holds one warp of each warpgroup
+// (warp w runs on sub-partition w % 4): two compute warps, one dQ warp and
+// one of the producer / MMA / idle warpgroup.
+constexpr int kBLaunchRegs = 128;
+constexpr int kBRegsCompute = 136;
+constexpr int kBRegsDq = 120;
+constexpr int kBRegsOther = 120;
+static_assert(2 * kBRegsCompute + kBRegsDq + kBRegsOther <= 4 * kBLaunchRegs,
+              "register split exceeds a sub-partition's pool");
 
 template <int D>
 struct BwdLayout {
@@ -54,7 +60,12 @@ struct BwdLayout {
   static constexpr int kKV = kBlockN * D * 2;      // K or V tile bytes
   static constexpr int kQT = BR * D * 2;           // Q or dO tile bytes
   static constexpr int kDS = kBlockN * BR * 2;     // dS^T tile bytes
-  static constexpr int kStage = BR * D * 4;        // fp32 dQ staging bytes
+  // fp32 dQ staging.  d = 64: one padded row per query (272-byte pitch, so
+  // that the eight rows of a 16-byte store phase start on different banks),
+  // each row added to the accumulator by its own thread; d = 128: the
+  // [64 queries][128 dims] tile, contiguous, added with one bulk reduce.
+  static constexpr int kStgPitch = (D == 64) ? D * 4 + 16 : D * 4;
+  static constexpr int kStage = BR * kStgPitch;
   // K/V buffers: two at d = 64, so that the next unit's key/value tiles load
   // while the current unit runs (units of short sequences are a few
   // iterations long); the Q/dO ring is then 2 deep to stay within shared
@@ -230,12 +241,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(BAR(L::kDSFull), 256);
     mbar_init(BAR(L::kDSEmpty), 1);
     mbar_init(BAR(L::kDQFull), 1);
-    mbar_init(BAR(L::kDQEmpty), 256);
+    mbar_init(BAR(L::kDQEmpty), 128);
     mbar_init(BAR(L::kAccFull), 1);
     mbar_init(BAR(L::kAccEmpty), 256);
     mbar_init(BAR(L::kDrain), 1);
     mbar_init(BAR(L::kStgFree), 1);
-    mbar_init(BAR(L::kStgDone), 256);
+    mbar_init(BAR(L::kStgDone), 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -252,8 +263,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // accumulator come from the preparation kernel
   grid_dependency_wait();
   grid_dependents_launch();
-  if (warp >= 8) regs_dec<kBRegsNarrow>();
-  else regs_inc<kBRegsWide>();
+  if (warp >= kBProducerWarp) regs_dec<kBRegsOther>();
+  else if (warp >= kBDqWarp0) regs_dec<kBRegsDq>();
+  else regs_inc<kBRegsCompute>();
 
   if (warp == kBProducerWarp) {
     // ---------------------------------------------------------------- producer
@@ -262,8 +274,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
+      // K, V: read once per unit.  Q, dO: re-read by every unit of the head
+      // (the CTAs working on one head run at about the same pace, so the
+      // reuse is close in time); normal priority, so that they do not push
+      // the fp32 dQ accumulator, reduce-added by the same CTAs, out of L2.
       const uint64_t pol_kv = l2_policy_evict_first();
-      const uint64_t pol_q = l2_policy_evict_last();
+      const uint64_t pol_q = l2_policy_evict_normal();
       uint32_t unit_iter = 0, q_iter = 0, kv_issued = 0;
       bool ok = true;
       for (int k = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++k), ++unit_iter) {
@@ -408,13 +424,86 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_commit(BAR(L::kDrain));
       mbar_wait_drain(BAR(L::kDrain), 0, p.wait_limit_ns);
     }
+  } else if (warp >= kBDqWarp0 && warp < kBDqWarp0 + 4) {
+    // ------------------------------------------------------ dQ warpgroup
+    // Walks the same iterations as the MMA issuer.  For each dQ tile: read
+    // it from tensor memory (thread = tensor-memory lane: the query row at
+    // d = 64, the head dimension at d = 128), release the tensor-memory tile,
+    // write it to the fp32 staging buffer and add it into the accumulator
+    // (the softmax scale is applied once, when the accumulator is converted).
+    const int t = threadIdx.x - 32 * kBDqWarp0;    // 0..127 = tensor-memory lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    uint8_t* stage = gbase + L::kStgOff;
+    const uint32_t stage_s = base + L::kStgOff;
+    uint32_t dq_cnt = 0;
+    bool ok = true;
+    for (int k = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++k)) {
+      const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
+      IterWin iw;
+      for (int it = 0; it < bu.n_it; ++it) {
+        if (!bactive<D, SPARSE>(iw, p, bu, it)) continue;
+        const uint32_t phase = dq_cnt & 1;
+        ok = warp_all(mbar_wait(BAR(L::kDQFull), phase, wc));
+        if (!ok) break;
+        ++dq_cnt;
+        tc_fence_after();
+        uint32_t v[64];
+        tmem_ld32(tmem + lane_off + L::kColDQ, v);
+        tmem_ld32(tmem + lane_off + L::kColDQ + 32u, v + 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(BAR(L::kDQEmpty));
+        float* acc_tile = p.dq_acc + ((size_t)bu.qbh(it) * p.n_pad + (size_t)bu.qtile(it) * BR) * D;
+        if constexpr (D == 64) {
+          // row t of the [128 queries][64 dims] tile: this thread's own
+          // staging row and its own bulk reduce (no cross-thread handshake);
+          // its previous reduce must have finished reading the row
+          if (dq_cnt > 1) bulk_wait_read0();
+          uint8_t* row = stage + t * L::kStgPitch;
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            *reinterpret_cast<float4*>(row + 16 * c) =
+                make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]), __uint_as_float(v[4 * c + 2]),
+                            __uint_as_float(v[4 * c + 3]));
+          fence_async_smem();
+          bulk_reduce_add_f32(acc_tile + (size_t)t * D, stage_s + t * L::kStgPitch, D * 4);
+          bulk_commit();
+        } else {
+          // column t of the [64 queries][128 dims] tile; one thread adds the
+          // whole tile once all 128 have written it.  The warpgroup meets on
+          // mbarriers with bounded waits, so a warp that timed out cannot
+          // leave the others waiting.
+          if (t == 0) {
+            bulk_wait_read0();  // the previous reduce has finished reading the tile
+            mbar_arrive(BAR(L::kStgFree));
+          }
+          ok = warp_all(mbar_wait(BAR(L::kStgFree), phase, wc));
+          if (!ok) break;
+          float* st = reinterpret_cast<float*>(stage);
+#pragma unroll
+          for (int q = 0; q < 64; ++q) st[q * 128 + t] = __uint_as_float(v[q]);
+          fence_async_smem();
+          mbar_arrive(BAR(L::kStgDone));
+          bool good = true;
+          if (t == 0) {
+            good = mbar_wait(BAR(L::kStgDone), phase, wc);
+            if (good) {
+              bulk_reduce_add_f32(acc_tile, stage_s, L::kStage);
+              bulk_commit();
+            }
+          }
+          ok = warp_all(good);
+          if (!ok) break;
+        }
+      }
+    }
+    bulk_wait0();  // every reduce this thread issued has landed before the CTA exits
   } else if (warp < 8) {
     // ------------------------------------------------- compute warpgroups 0, 1
     // Both warpgroups run the same loop on their own half of each query tile
     // (queries [w*HALF, (w+1)*HALF)), thread = key = tensor-memory lane:
-    //   P^T half, arrive P; stage dQ of the previous iteration (half of its
-    //   columns), arrive dQ-empty; dS^T half, arrive dS.  At the end of a unit
-    //   each warpgroup writes half of the dims of dK and dV.
+    //   P^T half, arrive P; dS^T half, arrive dS.  At the end of a unit each
+    //   warpgroup writes half of the dims of dK and dV.
     const int w = warp >> 2;                       // 0 or 1
     const int key_in = threadIdx.x & 127;          // tensor-memory lane
     const int tid256 = threadIdx.x;                // 0..255 over both warpgroups
@@ -422,77 +511,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t tS = tmem + lane_off + L::kColS;
     const uint32_t tDP = tmem + lane_off + L::kColDP;
     const float sl2 = p.scale_log2;
-    float* stage = reinterpret_cast<float*>(gbase + L::kStgOff);
-    const uint32_t stage_s = base + L::kStgOff;
     constexpr int HALF = L::HALF;
     constexpr int NC = HALF / 32;                  // 32-column chunks per warpgroup
-    uint32_t q_iter = 0, s_cnt = 0, dp_cnt = 0, ds_cnt = 0, dq_cnt = 0, unit_iter = 0;
-    int pend_qbh = -1, pend_i = 0;                 // dQ tile waiting to be staged
+    uint32_t q_iter = 0, s_cnt = 0, dp_cnt = 0, ds_cnt = 0, unit_iter = 0;
     bool ok = true;
-
-    // Stage the pending dQ tile: read this warpgroup's 32 columns of it from
-    // tensor memory, write them into the fp32 staging tile, then one thread
-    // adds the whole tile into the global accumulator (the softmax scale is
-    // applied once, when the accumulator is converted).
-    auto stage_dq = [&]() -> bool {
-      // The two warpgroups meet on mbarriers with bounded waits, not on a
-      // named barrier: if one of them has given up on a timeout, the other
-      // must not wait for it forever.
-      const uint32_t sphase = dq_cnt & 1;
-      if (!warp_all(mbar_wait(BAR(L::kDQFull), sphase, wc))) return false;
-      ++dq_cnt;
-      tc_fence_after();
-      uint32_t v[32];
-      tmem_ld32(tmem + lane_off + L::kColDQ + 32u * w, v);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(BAR(L::kDQEmpty));
-      if (tid256 == 0) {
-        bulk_wait_read0();  // the previous reduce has finished reading the tile
-        mbar_arrive(BAR(L::kStgFree));
-      }
-      if (!warp_all(mbar_wait(BAR(L::kStgFree), sphase, wc))) return false;
-      if (D == 64) {
-        // lane = query key_in, columns = dims 32w..32w+31 of row key_in of the
-        // [128 queries][64 dims] tile; chunk positions rotated by key_in mod 8
-        // (static barrel shift of the registers) to spread banks.
-        const int rot = key_in & 7;
-#pragma unroll
-        for (int b = 1; b < 8; b <<= 1) {
-          if (rot & b) {
-            uint32_t tmp[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) tmp[e] = v[(e + 4 * b) & 31];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = tmp[e];
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int ch = 8 * w + ((e + key_in) & 7);
-          float4 f = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                 __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
-          *reinterpret_cast<float4*>(stage + key_in * 64 + 4 * ch) = f;
-        }
-      } else {
-        // lane = dim key_in, columns = queries 32w..32w+31: column key_in of
-        // the [64 queries][128 dims] tile
-#pragma unroll
-        for (int q = 0; q < 32; ++q) stage[(32 * w + q) * 128 + key_in] = __uint_as_float(v[q]);
-      }
-      fence_async_smem();
-      mbar_arrive(BAR(L::kStgDone));
-      bool good = true;
-      if (tid256 == 0) {
-        good = mbar_wait(BAR(L::kStgDone), sphase, wc);
-        if (good) {
-          bulk_reduce_add_f32(p.dq_acc + ((size_t)pend_qbh * p.n_pad + (size_t)pend_i * BR) * D, stage_s, L::kStage);
-          bulk_commit();
-        }
-      }
-      pend_qbh = -1;
-      return warp_all(good);
-    };
 
     for (int k = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++k), ++unit_iter) {
       const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
@@ -560,9 +582,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_before();
         const bool withhold = (p.debug_flags & 2) && unit_iter == 0 && q_iter == 0 && tid256 == 0;
         if (!withhold) mbar_arrive(BAR(L::kPFull));
-        // dQ of the previous iteration (its MMA was issued after the previous
-        // dS; its tensor-memory tile is reused by this iteration's dQ MMA)
-        if (pend_qbh >= 0 && !(ok = stage_dq())) break;
         // dS^T = P^T o (dP^T - D)
         ok = warp_all(mbar_wait(BAR(L::kDPFull), dp_cnt & 1, wc));
         if (!ok) break;
@@ -620,8 +639,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(L::kDSFull));
-        pend_qbh = bu.qbh(it);
-        pend_i = i;
         ++q_iter;
         ++n_done;
       }
@@ -661,8 +678,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_before();
       mbar_arrive(BAR(L::kAccEmpty));
     }
-    if (ok && pend_qbh >= 0) stage_dq();  // the CTA's last dQ tile
-    if (tid256 == 0) bulk_wait0();        // every dQ reduce has landed before the CTA exits
   }
 
   __syncwarp();
