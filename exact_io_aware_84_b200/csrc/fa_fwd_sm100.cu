@@ -71,7 +71,12 @@ struct FwdLayout {
   static constexpr int kPVDone = kSFree + 2;     // [2]
   static constexpr int kDrain = kPVDone + 2;
   static constexpr int kNumBars = kDrain + 1;
-  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  // epilogue: per softmax warp a 32-row x 64-byte staging buffer (16-byte
+  // chunks XOR-swizzled by row), through which O is stored 8 rows x 64
+  // contiguous bytes per store instruction
+  static constexpr int kEpiWarpBytes = 32 * 64;
+  static constexpr int kEpiOff = (kBarOff + kNumBars * 8 + 127) / 128 * 128;
+  static constexpr int kMiscOff = kEpiOff + 8 * kEpiWarpBytes;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B
   // tensor-memory columns
@@ -683,8 +688,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (!ok) break;
       // ---- epilogue: O / l -> dtype -> global; LSE = (m + log2 l) ln 2.
-      // A row with no kept key (block-sparse) gets O = 0 and LSE = -inf; a
-      // tile that visits no key block at all skips tensor memory entirely.
+      // O is read from tensor memory 32 columns at a time, normalised,
+      // converted and stored through this warp's staging buffer, so that
+      // each store instruction writes 64 contiguous bytes of 8 rows (not 16
+      // bytes of 32 rows).  A row with no kept key (block-sparse) gets O = 0
+      // and LSE = -inf; a tile that visits no key block at all skips tensor
+      // memory entirely.
       if (nb > 0) {
         ok = warp_all(mbar_wait(BAR(L::kOFull + t), o_cnt & 1, wc));
         if (!ok) break;
@@ -692,43 +701,53 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_fence_after();
       }
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-      const bool in_range = row < p.N;
-      constexpr int kOBytes = O32 ? 4 : 2;
-      uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + ((size_t)ui.bh * p.N + (size_t)(in_range ? row : 0)) * D * kOBytes;
+      {
+        constexpr int kOBytes = O32 ? 4 : 2;
+        constexpr int kGroups = O32 ? 2 : 1;        // 64-byte groups per 32 columns
+        const int lane = threadIdx.x & 31;
+        uint8_t* stg = gbase + L::kEpiOff + warp * L::kEpiWarpBytes;
+        const int row0 = ui.r0(t) + (r_in & ~31);   // first row of this warp's 32
+        uint8_t* obase = reinterpret_cast<uint8_t*>(p.o) + (size_t)ui.bh * p.N * D * kOBytes;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        if (nb > 0) {
-          tmem_ld32(tO + 32u * c, o);
-          tmem_wait_ld();
-        } else {
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          if (nb > 0) {
+            tmem_ld32(tO + 32u * c, o);
+            tmem_wait_ld();
+          } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
-        }
-        if constexpr (FP8) {  // V's per-channel dequantisation scales
-          const float* svp = p.fp8_sv + (size_t)ui.kvbh * D + 32 * c;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * svp[e]);
-        }
-        if constexpr (O32) {
-          if (in_range) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 128);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              dst[e] = make_uint4(__float_as_uint(__uint_as_float(o[4 * e]) * inv_l),
-                                  __float_as_uint(__uint_as_float(o[4 * e + 1]) * inv_l),
-                                  __float_as_uint(__uint_as_float(o[4 * e + 2]) * inv_l),
-                                  __float_as_uint(__uint_as_float(o[4 * e + 3]) * inv_l));
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
           }
-        } else {
-          uint32_t w[16];
+          if constexpr (FP8) {  // V's per-channel dequantisation scales
+            const float* svp = p.fp8_sv + (size_t)ui.kvbh * D + 32 * c;
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            w[e] = pack2<BF16>(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-          if (in_range) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * svp[e]);
+          }
 #pragma unroll
-            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          for (int gi = 0; gi < kGroups; ++gi) {
+            uint32_t w[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              if constexpr (O32) w[e] = __float_as_uint(__uint_as_float(o[16 * gi + e]) * inv_l);
+              else w[e] = pack2<BF16>(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+            }
+            // this row's 64 bytes -> row `lane` of the staging buffer, chunk k
+            // at position k ^ ((row >> 1) & 3): the row-wise writes and the
+            // 8-rows x 4-chunks reads below are both free of bank conflicts
+            __syncwarp();
+#pragma unroll
+            for (int kc = 0; kc < 4; ++kc)
+              *reinterpret_cast<uint4*>(stg + lane * 64 + ((kc ^ ((lane >> 1) & 3)) * 16)) =
+                  make_uint4(w[4 * kc], w[4 * kc + 1], w[4 * kc + 2], w[4 * kc + 3]);
+            __syncwarp();
+            const int colb = (c * kGroups + gi) * 64;   // byte offset of the group within a row
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int rr = (lane >> 2) + 8 * i, kc = lane & 3;
+              const uint4 val = *reinterpret_cast<const uint4*>(stg + rr * 64 + ((kc ^ ((rr >> 1) & 3)) * 16));
+              if (row0 + rr < p.N)
+                *reinterpret_cast<uint4*>(obase + (size_t)(row0 + rr) * D * kOBytes + colb + kc * 16) = val;
+            }
           }
         }
       }
@@ -736,7 +755,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_fence_before();
         mbar_arrive(BAR(L::kOEmpty + t));
       }
-      if (in_range)
+      if (row < p.N)
         p.lse[(size_t)ui.bh * p.N + row] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
     }
   }
