@@ -37,9 +37,9 @@ def test_events_bracket_the_main_kernel_and_clear():
     torch.cuda.synchronize()
     assert fa.fa_last_device_status() == fa.FA_OK
     main_ms, call_ms = kb.elapsed_time(ka), outer_s.elapsed_time(outer_e)
-    # the main kernel lies inside the call and is most of it
-    assert 0.0 < main_ms <= call_ms
-    assert main_ms >= 0.5 * call_ms, (main_ms, call_ms)
+    # the main kernel lies inside the call (which also spans the other two
+    # launches and the host's work between the events)
+    assert 0.0 < main_ms <= call_ms, (main_ms, call_ms)
     for a, r in zip(got, ref):
         assert rel_fro(to64(a), to64(r)) < 1e-3
     # cleared: a later call leaves the events where they were
