@@ -23,11 +23,11 @@
 // S^T | dP^T | dV | dK | dQ fit in the 512 tensor-memory columns (448 used).
 // Roles (512 threads):
 //   warps 0-7   two compute warpgroups (thread = key = TMEM lane), each owning
-//               half of every query tile's columns: P^T, then dS^T; at the
-//               end of a unit each writes half of the head dims of dK and dV
+//               half of every query tile's columns: P^T, then dS^T
 //   warps 8-11  dQ warpgroup: drains each query tile's dQ from tensor memory
 //               into shared memory and adds it into the fp32 accumulator
-//               with bulk reduce-adds, concurrently with the compute warps
+//               with bulk reduce-adds, concurrently with the compute warps;
+//               at the end of a unit it writes the key tile's dK and dV
 //   warp  12    TMA producer      warp 13  MMA issuer      warps 14-15 idle
 #include <cuda_fp16.h>
 
@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(BAR(L::kDQFull), 1);
     mbar_init(BAR(L::kDQEmpty), 128);
     mbar_init(BAR(L::kAccFull), 1);
-    mbar_init(BAR(L::kAccEmpty), 256);
+    mbar_init(BAR(L::kAccEmpty), 128);
     mbar_init(BAR(L::kDrain), 1);
     mbar_init(BAR(L::kStgFree), 1);
     mbar_init(BAR(L::kStgDone), 128);
@@ -418,6 +418,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           ++q_iter;
         }
         if (!ok) break;
+        // A unit with no computed iteration never waited for the previous
+        // unit's accumulators to be read; wait here, so that the accumulator
+        // barrier is never two phases ahead of the warpgroup that reads it.
+        if (a0 >= bu.n_it && unit_iter > 0 && !mbar_wait(BAR(L::kAccEmpty), (unit_iter - 1) & 1, wc)) {
+          ok = false;
+          break;
+        }
         tc_commit(BAR(L::kAccFull));
         tc_commit(BAR(L::kKVEmpty + kb));
       }
@@ -435,13 +442,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     uint8_t* stage = gbase + L::kStgOff;
     const uint32_t stage_s = base + L::kStgOff;
-    uint32_t dq_cnt = 0;
+    uint32_t dq_cnt = 0, unit_iter = 0;
     bool ok = true;
-    for (int k = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++k)) {
+    for (int k = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++k), ++unit_iter) {
       const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
       IterWin iw;
+      int n_done = 0;  // iterations computed in this unit
       for (int it = 0; it < bu.n_it; ++it) {
         if (!bactive<D, SPARSE>(iw, p, bu, it)) continue;
+        ++n_done;
         const uint32_t phase = dq_cnt & 1;
         ok = warp_all(mbar_wait(BAR(L::kDQFull), phase, wc));
         if (!ok) break;
@@ -496,6 +505,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!ok) break;
         }
       }
+      if (!ok) break;
+      // dK, dV of this key tile (lane t = key): read from tensor memory once
+      // the unit's last products are done, then released to the next unit's
+      // first dV / dK products.  Done here rather than in the compute
+      // warpgroups, which go straight on to the next unit's first P.
+      ok = warp_all(mbar_wait(BAR(L::kAccFull), unit_iter & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      const int key = bu.jk * kBlockN + t;
+      const bool in_range = key < p.N;
+      const size_t rowoff = ((size_t)bu.kvbh * p.N + (size_t)(in_range ? key : 0)) * D * 2;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which ? L::kColDK : L::kColDV;
+        const float mul = which ? p.scale : 1.f;
+        uint8_t* dst = reinterpret_cast<uint8_t*>(which ? p.dk : p.dv) + rowoff;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          if (n_done > 0) {
+            tmem_ld32(tmem + lane_off + col + 32u * c, r);
+            tmem_wait_ld();
+          } else {  // no query attends this key tile: zero gradient
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = 0u;
+          }
+          if (which == 1 && c == D / 32 - 1) {  // every accumulator column has been read
+            tc_fence_before();
+            mbar_arrive(BAR(L::kAccEmpty));
+          }
+          uint32_t wv[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            wv[e] = pack2<BF16>(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
+          if (in_range) {
+            uint4* o = reinterpret_cast<uint4*>(dst + c * 64);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+          }
+        }
+      }
     }
     bulk_wait0();  // every reduce this thread issued has landed before the CTA exits
   } else if (warp < 8) {
@@ -520,7 +570,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
       const int key = bu.jk * kBlockN + key_in;
       const bool key_ok = key < p.N;
-      int n_done = 0;  // iterations computed in this unit
       IterWin iw;
       for (int it = 0; it < bu.n_it; ++it) {
         if (!bactive<D, SPARSE>(iw, p, bu, it)) continue;
@@ -640,43 +689,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_before();
         mbar_arrive(BAR(L::kDSFull));
         ++q_iter;
-        ++n_done;
       }
-      if (!ok) break;
-      // dK, dV of this key tile: lane = key, this warpgroup's half of the dims
-      ok = warp_all(mbar_wait(BAR(L::kAccFull), unit_iter & 1, wc));
-      if (!ok) break;
-      tc_fence_after();
-      const bool in_range = key < p.N;
-      const size_t rowoff = ((size_t)bu.kvbh * p.N + (size_t)(in_range ? key : 0)) * D * 2;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t col = (which ? L::kColDK : L::kColDV) + (uint32_t)(D / 2) * w;
-        const float mul = which ? p.scale : 1.f;
-        uint8_t* dst = reinterpret_cast<uint8_t*>(which ? p.dk : p.dv) + rowoff + (D / 2) * 2 * w;
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          uint32_t r[32];
-          if (n_done > 0) {
-            tmem_ld32(tmem + lane_off + col + 32u * c, r);
-            tmem_wait_ld();
-          } else {  // no query attends this key tile: zero gradient
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = 0u;
-          }
-          uint32_t wv[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            wv[e] = pack2<BF16>(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
-          if (in_range) {
-            uint4* o = reinterpret_cast<uint4*>(dst + c * 64);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) o[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(BAR(L::kAccEmpty));
     }
   }
 
