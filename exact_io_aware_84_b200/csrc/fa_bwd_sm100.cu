@@ -74,6 +74,14 @@ struct BwdLayout {
   static constexpr int kKOff = 0;                  // buffer b: K at b * 2 kKV, V after it
   static constexpr int kVOff = kKOff + kKV;
   static constexpr int kStages = (D == 64) ? 2 : 3;  // Q / dO / LSE / D ring depth
+  // d = 128 (3-deep ring): the MMA issuer's per-tile waits are folded into
+  // the two it must make anyway.  kPFull also means "the next tile's Q/dO
+  // have landed" (the compute warpgroups wait for them first) and kDSFull
+  // also means "dQ of the previous tile has left tensor memory" (the dQ
+  // warpgroup arrives on it).  With the 2-deep ring of d = 64 the next tile
+  // is often still loading when P is ready, so there the issuer waits on
+  // kQFull and kDQEmpty itself.
+  static constexpr bool kFoldWaits = (D == 128);
   static constexpr int kQOff = kKVBufs * 2 * kKV;    // [kStages]
   static constexpr int kDOOff = kQOff + kStages * kQT;
   static constexpr int kDSOff = kDOOff + kStages * kQT;
@@ -238,10 +246,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(BAR(L::kSFull), 1);
     mbar_init(BAR(L::kDPFull), 1);
     mbar_init(BAR(L::kPFull), 256);
-    mbar_init(BAR(L::kDSFull), 256);
+    // dS^T of tile i written (256 compute threads) and, folded, dQ of tile
+    // i-1 read out of tensor memory (128 dQ-warpgroup threads)
+    mbar_init(BAR(L::kDSFull), L::kFoldWaits ? 384 : 256);
+    mbar_init(BAR(L::kDQEmpty), 128);
     mbar_init(BAR(L::kDSEmpty), 1);
     mbar_init(BAR(L::kDQFull), 1);
-    mbar_init(BAR(L::kDQEmpty), 128);
     mbar_init(BAR(L::kAccFull), 1);
     mbar_init(BAR(L::kAccEmpty), 128);
     mbar_init(BAR(L::kDrain), 1);
@@ -382,11 +392,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int ks = 0; ks < BR / 16; ++ks)
             mma_ts(tmem + L::kColDV, tmem + L::kColS + L::packed_col(ks), sdesc_advance(dDOmn, mnmaj_off(ks)), idesc_acc,
                    (!first || ks > 0) ? 1u : 0u);
-          // S^T for the next query tile (the S region's P^T was consumed by dV above)
+          // S^T for the next query tile (the S region's P^T was consumed by dV
+          // above).  Folded: its Q tile has landed, since the compute
+          // warpgroups waited for it before arriving on kPFull.
           if (nxt < bu.n_it) {
             const uint32_t st1 = (q_iter + 1) % L::kStages;
-            if (!mbar_wait(BAR(L::kQFull + st1), ((q_iter + 1) / L::kStages) & 1, wc)) { ok = false; break; }
-            tc_fence_after();
+            if constexpr (!L::kFoldWaits) {
+              if (!mbar_wait(BAR(L::kQFull + st1), ((q_iter + 1) / L::kStages) & 1, wc)) { ok = false; break; }
+              tc_fence_after();
+            }
             const uint64_t dQ1 = kmaj<BR>(base + L::kQOff + st1 * L::kQT, 0);
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks)
@@ -402,9 +416,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int ks = 0; ks < BR / 16; ++ks)
             mma_ts(tmem + L::kColDK, tmem + L::kColDP + L::packed_col(ks), sdesc_advance(dQmn, mnmaj_off(ks)), idesc_acc,
                    (!first || ks > 0) ? 1u : 0u);
-          // dQ_i (d=64) or dQ_i^T (d=128) from dS^T in shared memory
-          if (dq_cnt > 0 && !mbar_wait(BAR(L::kDQEmpty), (dq_cnt - 1) & 1, wc)) { ok = false; break; }
-          tc_fence_after();
+          // dQ_i (d=64) or dQ_i^T (d=128) from dS^T in shared memory, once
+          // the dQ warpgroup has read dQ_{i-1} out of tensor memory (folded:
+          // before its arrival on kDSFull)
+          if constexpr (!L::kFoldWaits) {
+            if (dq_cnt > 0 && !mbar_wait(BAR(L::kDQEmpty), (dq_cnt - 1) & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+          }
 #pragma unroll
           for (int ks = 0; ks < kBlockN / 16; ++ks) {
             const uint64_t a = sdesc_advance(D == 64 ? dDSmn : dKmn, mnmaj_off(ks));
@@ -444,6 +462,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t stage_s = base + L::kStgOff;
     uint32_t dq_cnt = 0, unit_iter = 0;
     bool ok = true;
+    // Folded waits: the dQ tensor-memory tile is free for the first dQ
+    // product, this warpgroup's share of the first kDSFull phase.  Each later
+    // arrival (after dQ_i is read out) belongs to the phase of tile i+1,
+    // which cannot begin before the issuer has consumed tile i's phase.
+    if constexpr (L::kFoldWaits) mbar_arrive(BAR(L::kDSFull));
     for (int k = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++k), ++unit_iter) {
       const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
       IterWin iw;
@@ -461,7 +484,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(tmem + lane_off + L::kColDQ + 32u, v + 32);
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(BAR(L::kDQEmpty));
+        mbar_arrive(BAR(L::kFoldWaits ? L::kDSFull : L::kDQEmpty));
         float* acc_tile = p.dq_acc + ((size_t)bu.qbh(it) * p.n_pad + (size_t)bu.qtile(it) * BR) * D;
         if constexpr (D == 64) {
           // row t of the [128 queries][64 dims] tile: this thread's own
@@ -571,12 +594,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int key = bu.jk * kBlockN + key_in;
       const bool key_ok = key < p.N;
       IterWin iw;
+      bool q_seen = false;  // this tile's Q/dO stage was already waited for
       for (int it = 0; it < bu.n_it; ++it) {
         if (!bactive<D, SPARSE>(iw, p, bu, it)) continue;
         const int i = bu.qtile(it);
         const uint32_t st = q_iter % L::kStages;
-        ok = warp_all(mbar_wait(BAR(L::kQFull + st), (q_iter / L::kStages) & 1, wc));
-        if (!ok) break;
+        if (!q_seen) {
+          ok = warp_all(mbar_wait(BAR(L::kQFull + st), (q_iter / L::kStages) & 1, wc));
+          if (!ok) break;
+        }
         // this half's -LSE*log2e and D, read four at a time (16-byte aligned)
         const float4* nlse2 = reinterpret_cast<const float4*>(gbase + L::kVecOff + st * L::kVecStage) + HALF * w / 4;
         const float4* dvec = nlse2 + BR / 4;
@@ -629,6 +655,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int c = 0; c < NC; ++c) tmem_st16(tS + HALF * w + 16u * c, pk + 16 * c);
         tmem_wait_st();
         tc_fence_before();
+        // Folded waits: the issuer computes the next tile's S^T right after
+        // dV; wait here for that tile's Q, so the issuer needs no wait of its
+        // own.  (The scan moves the mask window forward; the loop's own test
+        // of the next iterations then refetches it.)
+        if constexpr (L::kFoldWaits) {
+          int nxt = it + 1;
+          while (nxt < bu.n_it && !bactive<D, SPARSE>(iw, p, bu, nxt)) ++nxt;
+          q_seen = nxt < bu.n_it;
+        }
+        if (q_seen) {
+          const uint32_t q1 = q_iter + 1;
+          ok = warp_all(mbar_wait(BAR(L::kQFull + q1 % L::kStages), (q1 / L::kStages) & 1, wc));
+          if (!ok) break;
+        }
         const bool withhold = (p.debug_flags & 2) && unit_iter == 0 && q_iter == 0 && tid256 == 0;
         if (!withhold) mbar_arrive(BAR(L::kPFull));
         // dS^T = P^T o (dP^T - D)
