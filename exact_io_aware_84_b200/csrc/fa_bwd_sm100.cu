@@ -344,7 +344,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       constexpr uint32_t idesc_acc = make_idesc_f16(BF16, kBlockN, D, false, true);   // dV, dK
       // dQ (d=64: M=128 queries, N=64) or dQ^T (d=128: M=128 dims, N=64 queries)
       constexpr uint32_t idesc_dq = make_idesc_f16(BF16, 128, 64, true, true);
-      uint32_t unit_iter = 0, q_iter = 0, p_cnt = 0, ds_cnt = 0, dq_cnt = 0;
+      uint32_t unit_iter = 0, p_cnt = 0, ds_cnt = 0, dq_cnt = 0;
+      // The issuer runs barely ahead of the tensor core, so its bookkeeping
+      // between products is kept short: the Q/dO descriptors of ring stage
+      // s are stage 0's advanced by s * kQT bytes, and the stage index and
+      // its phase are stepped, not divided out of a tile counter.
+      const uint64_t dQ0 = kmaj<BR>(base + L::kQOff, 0), dDO0 = kmaj<BR>(base + L::kDOOff, 0);
+      const uint64_t dQmn0 = mnmaj<BR>(base + L::kQOff, 0), dDOmn0 = mnmaj<BR>(base + L::kDOOff, 0);
+      uint32_t st = 0, st_ph = 0;  // ring stage of the current tile and the parity of its use
+      auto next_stage = [](uint32_t s0, uint32_t ph0, uint32_t& s1, uint32_t& ph1) {
+        s1 = s0 + 1 == (uint32_t)L::kStages ? 0u : s0 + 1;
+        ph1 = s1 == 0 ? ph0 ^ 1u : ph0;
+      };
       bool ok = true;
       for (int k = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++k), ++unit_iter) {
         const BUnit bu = decode_bunit<D, CAUSAL>(u, p);
@@ -358,10 +369,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         while (a0 < bu.n_it && !bactive<D, SPARSE>(iw, p, bu, a0)) ++a0;
         // S^T for the first query tile
         if (a0 < bu.n_it) {
-          const uint32_t st = q_iter % L::kStages;
-          if (!mbar_wait(BAR(L::kQFull + st), (q_iter / L::kStages) & 1, wc)) { ok = false; break; }
+          if (!mbar_wait(BAR(L::kQFull + st), st_ph, wc)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t dQ = kmaj<BR>(base + L::kQOff + st * L::kQT, 0);
+          const uint64_t dQ = sdesc_advance(dQ0, st * L::kQT);
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks)
             mma_ss(tmem + L::kColS, sdesc_advance(dK, kmaj_off<kBlockN>(ks)), sdesc_advance(dQ, kmaj_off<BR>(ks)),
@@ -369,10 +379,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_commit(BAR(L::kSFull));
         }
         for (int it = a0, nxt; it < bu.n_it; it = nxt) {  // active iterations only
-          const uint32_t st = q_iter % L::kStages;
-          const uint32_t sQ = base + L::kQOff + st * L::kQT;
-          const uint32_t sDO = base + L::kDOOff + st * L::kQT;
-          const uint64_t dDO = kmaj<BR>(sDO, 0), dDOmn = mnmaj<BR>(sDO, 0), dQmn = mnmaj<BR>(sQ, 0);
+          const uint32_t soff = st * L::kQT;
+          const uint64_t dDO = sdesc_advance(dDO0, soff), dDOmn = sdesc_advance(dDOmn0, soff),
+                         dQmn = sdesc_advance(dQmn0, soff);
+          uint32_t st1, st1_ph;  // stage of the next tile
+          next_stage(st, st_ph, st1, st1_ph);
           const uint32_t first = (it == a0);
           nxt = it + 1;
           while (nxt < bu.n_it && !bactive<D, SPARSE>(iw, p, bu, nxt)) ++nxt;
@@ -396,12 +407,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           // above).  Folded: its Q tile has landed, since the compute
           // warpgroups waited for it before arriving on kPFull.
           if (nxt < bu.n_it) {
-            const uint32_t st1 = (q_iter + 1) % L::kStages;
             if constexpr (!L::kFoldWaits) {
-              if (!mbar_wait(BAR(L::kQFull + st1), ((q_iter + 1) / L::kStages) & 1, wc)) { ok = false; break; }
+              if (!mbar_wait(BAR(L::kQFull + st1), st1_ph, wc)) { ok = false; break; }
               tc_fence_after();
             }
-            const uint64_t dQ1 = kmaj<BR>(base + L::kQOff + st1 * L::kQT, 0);
+            const uint64_t dQ1 = sdesc_advance(dQ0, st1 * L::kQT);
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks)
               mma_ss(tmem + L::kColS, sdesc_advance(dK, kmaj_off<kBlockN>(ks)), sdesc_advance(dQ1, kmaj_off<BR>(ks)),
@@ -433,7 +443,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           ++dq_cnt;
           tc_commit(BAR(L::kDSEmpty));       // dS^T shared tile no longer read
           tc_commit(BAR(L::kQEmpty + st));   // Q_i, dO_i, LSE_i, D_i no longer read
-          ++q_iter;
+          st = st1;
+          st_ph = st1_ph;
         }
         if (!ok) break;
         // A unit with no computed iteration never waited for the previous
