@@ -57,8 +57,12 @@ def test_small_shapes_fp16(d, causal):
     _check_heads(w, x, grads)
 
 
-def test_many_units_per_cta():
-    w = Workload("many", 3, 64, 384, 64, "bf16", True, 0.125, True, seed=5)
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("d", [64, 128])
+def test_many_units_per_cta(d, causal):
+    # several units per CTA: the barrier phases carried across units (and at
+    # d = 128 the issuer's waits folded into the P and dS barriers)
+    w = Workload("many", 3, 64, 384, d, "bf16", causal, 1.0 / d ** 0.5, True, seed=5 + d)
     x, g, grads = _run(w)
     _check_heads(w, x, grads, pairs=[(0, 0), (1, 31), (2, 63)])
 
