@@ -29,6 +29,10 @@
 //               with bulk reduce-adds, concurrently with the compute warps;
 //               at the end of a unit it writes the key tile's dK and dV
 //   warp  12    TMA producer      warp 13  MMA issuer      warps 14-15 idle
+// The issuer runs barely ahead of the tensor core, so each of its waits and
+// each piece of its bookkeeping leaves the tensor core idle: per query tile
+// it waits only for P (before dV) and dS (before dK, dQ) at d = 128, the
+// other two conditions being folded into those barriers (kFoldWaits).
 #include <cuda_fp16.h>
 
 #include <type_traits>
