@@ -86,6 +86,16 @@ struct BwdLayout {
   // is often still loading when P is ready, so there the issuer waits on
   // kQFull and kDQEmpty itself.
   static constexpr bool kFoldWaits = (D == 128);
+  // d = 128: two MMA issuers, so that one issues while the other waits.
+  // Issuer A (warp 13) owns the dP region and the dK / dQ accumulators
+  // (dP, dK, dQ; waits on kDSFull), issuer B (warp 14) the S region and dV
+  // (S, dV; waits on kPFull).  Their products touch disjoint tensor-memory
+  // columns, so the tensor core may interleave the two streams in any order;
+  // within each stream a thread's MMAs run in issue order.  Barriers that
+  // both streams release (Q/dO stage, K/V tiles, accumulators, drain) count
+  // one commit per issuer.
+  static constexpr bool kTwoIssuers = kFoldWaits;
+  static constexpr int kIssuers = kTwoIssuers ? 2 : 1;
   static constexpr int kQOff = kKVBufs * 2 * kKV;    // [kStages]
   static constexpr int kDOOff = kQOff + kStages * kQT;
   static constexpr int kDSOff = kDOOff + kStages * kQT;
@@ -241,11 +251,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (threadIdx.x == 0) {
     for (int b = 0; b < L::kKVBufs; ++b) {
       mbar_init(BAR(L::kKVFull + b), 1);
-      mbar_init(BAR(L::kKVEmpty + b), 1);
+      mbar_init(BAR(L::kKVEmpty + b), L::kIssuers);
     }
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(BAR(L::kQFull + s), 1);
-      mbar_init(BAR(L::kQEmpty + s), 1);
+      mbar_init(BAR(L::kQEmpty + s), L::kIssuers);
     }
     mbar_init(BAR(L::kSFull), 1);
     mbar_init(BAR(L::kDPFull), 1);
@@ -256,9 +266,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(BAR(L::kDQEmpty), 128);
     mbar_init(BAR(L::kDSEmpty), 1);
     mbar_init(BAR(L::kDQFull), 1);
-    mbar_init(BAR(L::kAccFull), 1);
+    mbar_init(BAR(L::kAccFull), L::kIssuers);
     mbar_init(BAR(L::kAccEmpty), 128);
-    mbar_init(BAR(L::kDrain), 1);
+    mbar_init(BAR(L::kDrain), L::kIssuers);
     mbar_init(BAR(L::kStgFree), 1);
     mbar_init(BAR(L::kStgDone), 128);
     *abort_flag = 0;
@@ -341,8 +351,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
     }
-  } else if (warp == kBMmaWarp) {
+  } else if (warp == kBMmaWarp || (L::kTwoIssuers && warp == kBMmaWarp + 1)) {
     // ---------------------------------------------------------------- MMA
+    // role 0: the single issuer (d = 64); 1: issuer A (dP, dK, dQ); 2: issuer
+    // B (S, dV)
+    const int role = L::kTwoIssuers ? (warp == kBMmaWarp ? 1 : 2) : 0;
+    const bool do_a = role != 2, do_b = role != 1;
     if (lane == 0) {
       constexpr uint32_t idesc_s = make_idesc_f16(BF16, kBlockN, BR, false, false);   // S^T, dP^T
       constexpr uint32_t idesc_acc = make_idesc_f16(BF16, kBlockN, D, false, true);   // dV, dK
@@ -371,16 +385,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         IterWin iw;  // walks forward only: the scan for the next iteration leads
         int a0 = 0;  // first computed iteration (n_it when the key tile is attended by none)
         while (a0 < bu.n_it && !bactive<D, SPARSE>(iw, p, bu, a0)) ++a0;
-        // S^T for the first query tile
+        // S^T (and, issuer A, dP^T) for the first query tile
         if (a0 < bu.n_it) {
           if (!mbar_wait(BAR(L::kQFull + st), st_ph, wc)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t dQ = sdesc_advance(dQ0, st * L::kQT);
+          if (do_b) {
+            const uint64_t dQ = sdesc_advance(dQ0, st * L::kQT);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            mma_ss(tmem + L::kColS, sdesc_advance(dK, kmaj_off<kBlockN>(ks)), sdesc_advance(dQ, kmaj_off<BR>(ks)),
-                   idesc_s, ks > 0);
-          tc_commit(BAR(L::kSFull));
+            for (int ks = 0; ks < D / 16; ++ks)
+              mma_ss(tmem + L::kColS, sdesc_advance(dK, kmaj_off<kBlockN>(ks)), sdesc_advance(dQ, kmaj_off<BR>(ks)),
+                     idesc_s, ks > 0);
+            tc_commit(BAR(L::kSFull));
+          }
+          if (role == 1) {
+            const uint64_t dDO = sdesc_advance(dDO0, st * L::kQT);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks)
+              mma_ss(tmem + L::kColDP, sdesc_advance(dV, kmaj_off<kBlockN>(ks)), sdesc_advance(dDO, kmaj_off<BR>(ks)),
+                     idesc_s, ks > 0);
+            tc_commit(BAR(L::kDPFull));
+          }
         }
         for (int it = a0, nxt; it < bu.n_it; it = nxt) {  // active iterations only
           const uint32_t soff = st * L::kQT;
@@ -391,13 +415,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const uint32_t first = (it == a0);
           nxt = it + 1;
           while (nxt < bu.n_it && !bactive<D, SPARSE>(iw, p, bu, nxt)) ++nxt;
-          // dP^T = V_j dO_i^T   (the dP region's previous contents, dS^T of
-          // tile i-1, were consumed by dK(i-1), issued earlier)
+          if (role == 0) {
+            // dP^T = V_j dO_i^T   (the dP region's previous contents, dS^T
+            // of tile i-1, were consumed by dK(i-1), issued earlier)
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            mma_ss(tmem + L::kColDP, sdesc_advance(dV, kmaj_off<kBlockN>(ks)), sdesc_advance(dDO, kmaj_off<BR>(ks)),
-                   idesc_s, ks > 0);
-          tc_commit(BAR(L::kDPFull));
+            for (int ks = 0; ks < D / 16; ++ks)
+              mma_ss(tmem + L::kColDP, sdesc_advance(dV, kmaj_off<kBlockN>(ks)), sdesc_advance(dDO, kmaj_off<BR>(ks)),
+                     idesc_s, ks > 0);
+            tc_commit(BAR(L::kDPFull));
+          }
+          if (do_b) {
           // dV += P^T dO_i
           if (!mbar_wait(BAR(L::kPFull), p_cnt & 1, wc)) { ok = false; break; }
           ++p_cnt;
@@ -422,14 +449,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                      idesc_s, ks > 0);
             tc_commit(BAR(L::kSFull));
           }
+          }  // do_b
+          if (do_a) {
           if (!mbar_wait(BAR(L::kDSFull), ds_cnt & 1, wc)) { ok = false; break; }
           ++ds_cnt;
+          if (role == 1 && first && unit_iter > 0 && !mbar_wait(BAR(L::kAccEmpty), (unit_iter - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           // dK += dS^T Q_i
 #pragma unroll
           for (int ks = 0; ks < BR / 16; ++ks)
             mma_ts(tmem + L::kColDK, tmem + L::kColDP + L::packed_col(ks), sdesc_advance(dQmn, mnmaj_off(ks)), idesc_acc,
                    (!first || ks > 0) ? 1u : 0u);
+          if (role == 1 && nxt < bu.n_it) {
+            // dP^T of the next tile (after dK(i), the last reader of the dP
+            // region's dS^T; its dO has landed: the compute warpgroups waited
+            // for it before arriving on kPFull, and so before kDSFull)
+            const uint64_t dDO1 = sdesc_advance(dDO0, st1 * L::kQT);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks)
+              mma_ss(tmem + L::kColDP, sdesc_advance(dV, kmaj_off<kBlockN>(ks)), sdesc_advance(dDO1, kmaj_off<BR>(ks)),
+                     idesc_s, ks > 0);
+            tc_commit(BAR(L::kDPFull));
+          }
           // dQ_i (d=64) or dQ_i^T (d=128) from dS^T in shared memory, once
           // the dQ warpgroup has read dQ_{i-1} out of tensor memory (folded:
           // before its arrival on kDSFull)
@@ -446,7 +490,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_commit(BAR(L::kDQFull));
           ++dq_cnt;
           tc_commit(BAR(L::kDSEmpty));       // dS^T shared tile no longer read
-          tc_commit(BAR(L::kQEmpty + st));   // Q_i, dO_i, LSE_i, D_i no longer read
+          }  // do_a
+          tc_commit(BAR(L::kQEmpty + st));   // Q_i, dO_i, LSE_i, D_i no longer read (this issuer)
           st = st1;
           st_ph = st1_ph;
         }
