@@ -29,10 +29,13 @@
 //               with bulk reduce-adds, concurrently with the compute warps;
 //               at the end of a unit it writes the key tile's dK and dV
 //   warp  12    TMA producer      warp 13  MMA issuer      warps 14-15 idle
-// The issuer runs barely ahead of the tensor core, so each of its waits and
-// each piece of its bookkeeping leaves the tensor core idle: per query tile
-// it waits only for P (before dV) and dS (before dK, dQ) at d = 128, the
-// other two conditions being folded into those barriers (kFoldWaits).
+//   (d = 128: warp 13 issues dP, dK, dQ and warp 14 issues S, dV)
+// An issuer runs barely ahead of the tensor core, so each of its waits and
+// each piece of its bookkeeping leaves the tensor core idle.  At d = 128 the
+// products are split over two issuers with disjoint tensor-memory regions,
+// so one issues while the other waits, and each waits once per query tile
+// (A for dS, B for P), the other conditions being folded into those
+// barriers (kFoldWaits, kTwoIssuers).
 #include <cuda_fp16.h>
 
 #include <type_traits>
