@@ -102,7 +102,10 @@ struct BwdLayout {
   static constexpr int kQOff = kKVBufs * 2 * kKV;    // [kStages]
   static constexpr int kDOOff = kQOff + kStages * kQT;
   static constexpr int kDSOff = kDOOff + kStages * kQT;
-  static constexpr int kStgOff = kDSOff + kDS;
+  // d = 128 (two issuers): two dS^T shared tiles, so that the compute
+  // warpgroups write tile i's while dQ(i-1) still reads tile i-1's
+  static constexpr int kDSBufs = (D == 128) ? 2 : 1;
+  static constexpr int kStgOff = kDSOff + kDSBufs * kDS;
   static constexpr int kVecOff = kStgOff + kStage;  // [kStages] x (nlse2[BR], dvec[BR])
   static constexpr int kVecStage = 2 * BR * 4;
   static constexpr int kBarOff = kVecOff + kStages * kVecStage;
@@ -115,7 +118,8 @@ struct BwdLayout {
   static constexpr int kDQEmpty = kSFull + 6, kAccFull = kSFull + 7, kAccEmpty = kSFull + 8, kDrain = kSFull + 9;
   // dQ staging tile: free again (previous reduce has read it) / fully written
   static constexpr int kStgFree = kSFull + 10, kStgDone = kSFull + 11;
-  static constexpr int kNumBars = kStgDone + 1;
+  static constexpr int kDSEmpty1 = kSFull + 12;   // dS^T shared tile 1 read (two tiles)
+  static constexpr int kNumBars = kDSEmpty1 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -268,6 +272,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(BAR(L::kDSFull), L::kFoldWaits ? 384 : 256);
     mbar_init(BAR(L::kDQEmpty), 128);
     mbar_init(BAR(L::kDSEmpty), 1);
+    mbar_init(BAR(L::kDSEmpty1), 1);
     mbar_init(BAR(L::kDQFull), 1);
     mbar_init(BAR(L::kAccFull), L::kIssuers);
     mbar_init(BAR(L::kAccEmpty), 128);
@@ -384,7 +389,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!mbar_wait(BAR(L::kKVFull + kb), (unit_iter / L::kKVBufs) & 1, wc)) { ok = false; break; }
         const uint32_t sK = base + kb * 2 * L::kKV + L::kKOff, sV = base + kb * 2 * L::kKV + L::kVOff;
         const uint64_t dK = kmaj<kBlockN>(sK, 0), dV = kmaj<kBlockN>(sV, 0), dKmn = mnmaj<kBlockN>(sK, 0);
-        const uint64_t dDSmn = mnmaj<kBlockN>(base + L::kDSOff, 0);
+        const uint64_t dDSmn0 = mnmaj<kBlockN>(base + L::kDSOff, 0);
         IterWin iw;  // walks forward only: the scan for the next iteration leads
         int a0 = 0;  // first computed iteration (n_it when the key tile is attended by none)
         while (a0 < bu.n_it && !bactive<D, SPARSE>(iw, p, bu, a0)) ++a0;
@@ -455,6 +460,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }  // do_b
           if (do_a) {
           if (!mbar_wait(BAR(L::kDSFull), ds_cnt & 1, wc)) { ok = false; break; }
+          const uint32_t db = L::kDSBufs == 2 ? (ds_cnt & 1u) : 0u;   // dS^T shared tile of this query tile
+          const uint64_t dDSmn = sdesc_advance(dDSmn0, db * L::kDS);
           ++ds_cnt;
           if (role == 1 && first && unit_iter > 0 && !mbar_wait(BAR(L::kAccEmpty), (unit_iter - 1) & 1, wc)) {
             ok = false;
@@ -492,7 +499,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           tc_commit(BAR(L::kDQFull));
           ++dq_cnt;
-          tc_commit(BAR(L::kDSEmpty));       // dS^T shared tile no longer read
+          tc_commit(BAR(db ? L::kDSEmpty1 : L::kDSEmpty));   // dS^T shared tile db no longer read
           }  // do_a
           tc_commit(BAR(L::kQEmpty + st));   // Q_i, dO_i, LSE_i, D_i no longer read (this issuer)
           st = st1;
@@ -739,7 +746,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!ok) break;
         ++dp_cnt;
         tc_fence_after();
-        ok = warp_all(ds_cnt == 0 || mbar_wait(BAR(L::kDSEmpty), (ds_cnt - 1) & 1, wc));
+        // the dS^T shared tile this query tile writes has been read by its
+        // previous dQ product (two tiles: the one two query tiles back)
+        const uint32_t db = L::kDSBufs == 2 ? (ds_cnt & 1u) : 0u;
+        if constexpr (L::kDSBufs == 2)
+          ok = warp_all(ds_cnt < 2 || mbar_wait(BAR(db ? L::kDSEmpty1 : L::kDSEmpty), ((ds_cnt >> 1) - 1) & 1, wc));
+        else
+          ok = warp_all(ds_cnt == 0 || mbar_wait(BAR(L::kDSEmpty), (ds_cnt - 1) & 1, wc));
         if (!ok) break;
         ++ds_cnt;
         // dS^T chunk by chunk into tensor memory (for the dK MMA) and into the
@@ -747,7 +760,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // column block cb holds queries 64cb..64cb+63; 16-byte chunk ch of row
         // key_in lives at position ch ^ (key_in & 7).  Packed dS^T chunk c goes
         // to columns [HALF*w + 16c, +16): dP^T chunk c/2 of this half, read.
-        uint8_t* ds_tile = gbase + L::kDSOff;
+        uint8_t* ds_tile = gbase + L::kDSOff + db * L::kDS;
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
           uint32_t r[32];
