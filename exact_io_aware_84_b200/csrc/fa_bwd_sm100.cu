@@ -29,7 +29,8 @@
 //               with bulk reduce-adds, concurrently with the compute warps;
 //               at the end of a unit it writes the key tile's dK and dV
 //   warp  12    TMA producer      warp 13  MMA issuer      warps 14-15 idle
-//   (d = 128: warp 13 issues dP, dK, dQ and warp 14 issues S, dV)
+//   (d = 128: warp 13 issues dP, dK, dQ and warp 14 issues S, dV, with the
+//   unit's K tile copied into tensor memory as the A operand of S^T)
 // An issuer runs barely ahead of the tensor core, so each of its waits and
 // each piece of its bookkeeping leaves the tensor core idle.  At d = 128 the
 // products are split over two issuers with disjoint tensor-memory regions,
@@ -129,6 +130,10 @@ struct BwdLayout {
   static constexpr uint32_t kColDV = 2 * BR;
   static constexpr uint32_t kColDK = 2 * BR + D;
   static constexpr uint32_t kColDQ = 2 * BR + 2 * D;
+  // two issuers (d = 128): the unit's K tile is copied into the last 64
+  // columns, so that S^T reads only Q from shared memory
+  static constexpr uint32_t kColK = kColDQ + BR;
+  static_assert(!kFoldWaits || kColK + D / 2 <= 512, "tensor memory overflow");
   static_assert(kColDQ + (D == 64 ? D : BR) <= 512, "tensor memory overflow");
   // Compute warpgroup w (0, 1) owns query columns [w*HALF, (w+1)*HALF) of
   // each tile and packs its 16-bit P^T / dS^T (two per 32-bit column) at the
@@ -399,10 +404,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_fence_after();
           if (do_b) {
             const uint64_t dQ = sdesc_advance(dQ0, st * L::kQT);
+            if (role == 2) {
+              // K into tensor memory, one K step (128 keys x 16 dims) per copy;
+              // the previous unit's S^T products, issued earlier by this
+              // thread, have read the region before these copies run
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks)
-              mma_ss(tmem + L::kColS, sdesc_advance(dK, kmaj_off<kBlockN>(ks)), sdesc_advance(dQ, kmaj_off<BR>(ks)),
-                     idesc_s, ks > 0);
+              for (int ks = 0; ks < D / 16; ++ks)
+                tc_cp_128x256b(tmem + L::kColK + 8u * ks, sdesc_advance(dK, kmaj_off<kBlockN>(ks)));
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks)
+                mma_ts(tmem + L::kColS, tmem + L::kColK + 8u * ks, sdesc_advance(dQ, kmaj_off<BR>(ks)), idesc_s,
+                       ks > 0);
+            } else {
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks)
+                mma_ss(tmem + L::kColS, sdesc_advance(dK, kmaj_off<kBlockN>(ks)), sdesc_advance(dQ, kmaj_off<BR>(ks)),
+                       idesc_s, ks > 0);
+            }
             tc_commit(BAR(L::kSFull));
           }
           if (role == 1) {
@@ -451,10 +469,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               tc_fence_after();
             }
             const uint64_t dQ1 = sdesc_advance(dQ0, st1 * L::kQT);
+            if (role == 2) {
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks)
-              mma_ss(tmem + L::kColS, sdesc_advance(dK, kmaj_off<kBlockN>(ks)), sdesc_advance(dQ1, kmaj_off<BR>(ks)),
-                     idesc_s, ks > 0);
+              for (int ks = 0; ks < D / 16; ++ks)
+                mma_ts(tmem + L::kColS, tmem + L::kColK + 8u * ks, sdesc_advance(dQ1, kmaj_off<BR>(ks)), idesc_s,
+                       ks > 0);
+            } else {
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks)
+                mma_ss(tmem + L::kColS, sdesc_advance(dK, kmaj_off<kBlockN>(ks)), sdesc_advance(dQ1, kmaj_off<BR>(ks)),
+                       idesc_s, ks > 0);
+            }
             tc_commit(BAR(L::kSFull));
           }
           }  // do_b

@@ -215,6 +215,14 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// Copy a 128-row x 256-bit matrix (one 16-element K step of a 16-bit K-major
+// operand, as the shared-memory descriptor describes it, swizzle included)
+// into tensor memory: row r to lane r, 8 consecutive 32-bit columns.  Ordered
+// with the issuing thread's later tcgen05.mma.
+__device__ __forceinline__ void tc_cp_128x256b(uint32_t taddr, uint64_t s_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");
+}
+
 // Instruction descriptor for kind::f16 with fp32 accumulation.
 //   bits 4-5 D format (1 = f32), 7-9 A format, 10-12 B format (0 = f16,
 //   1 = bf16), 15 A major, 16 B major (0 = K-major, 1 = MN-major),
